@@ -1,0 +1,234 @@
+"""fp64 CPU oracle for exact attention forward (test infrastructure).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the package smoke check and the
+benchmark's CPU-baseline leg are the only code allowed to import this package.
+The CUDA product path never imports, links or calls it, and shares no code
+with it. The arithmetic lives in ``oracle.c`` (plain C, double precision, one
+materialised score row at a time); this module compiles it with gcc and
+marshals numpy arrays into it.
+
+Pins (tests/test_oracle.py): closed forms (one key, two keys, uniform scores
+-> mean of V and LSE = ln(count)), constant V, causal row 0, GQA equal to the
+repeat_kv-expanded MHA, mask counts and analytic tile classes, split
+invariance of the LSE combine, paging invariance, the ALiBi slope sequence for
+8 heads, and torch's fp64 CPU scaled_dot_product_attention on small cases.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+MASK_NONE, MASK_CAUSAL, MASK_WINDOW, MASK_DOCUMENT = 0, 1, 2, 3
+MOD_NONE, MOD_SOFTCAP, MOD_ALIBI = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (plain gcc, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-fno-fast-math", "-pthread",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _AttnArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("q_sb", ctypes.c_int64), ("q_ss", ctypes.c_int64), ("q_sh", ctypes.c_int64),
+        ("k_sb", ctypes.c_int64), ("k_ss", ctypes.c_int64), ("k_sh", ctypes.c_int64),
+        ("v_sb", ctypes.c_int64), ("v_ss", ctypes.c_int64), ("v_sh", ctypes.c_int64),
+        ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+        ("Sq", ctypes.c_int), ("Skv", ctypes.c_int), ("D", ctypes.c_int),
+        ("scale", ctypes.c_double),
+        ("mask", ctypes.c_int), ("window_left", ctypes.c_int), ("window_right", ctypes.c_int),
+        ("q_offset", ctypes.c_int),
+        ("doc_id", ctypes.c_void_p),
+        ("mod", ctypes.c_int), ("softcap", ctypes.c_double),
+        ("alibi", ctypes.c_void_p), ("alibi_bstride", ctypes.c_int64),
+        ("kv_begin", ctypes.c_int), ("kv_end", ctypes.c_int),
+    ]
+
+
+class _DecodeArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("q_sb", ctypes.c_int64), ("q_sh", ctypes.c_int64),
+        ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+        ("c_sp", ctypes.c_int64), ("c_ss", ctypes.c_int64), ("c_sh", ctypes.c_int64),
+        ("block_table", ctypes.c_void_p), ("bt_stride", ctypes.c_int64), ("seqlens", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("D", ctypes.c_int),
+        ("page_size", ctypes.c_int), ("num_pages", ctypes.c_int),
+        ("scale", ctypes.c_double), ("mod", ctypes.c_int), ("softcap", ctypes.c_double),
+        ("alibi", ctypes.c_void_p), ("alibi_bstride", ctypes.c_int64),
+    ]
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oracle_attn.argtypes = [ctypes.POINTER(_AttnArgs), ctypes.c_void_p, ctypes.c_int64,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+            lib.oracle_attn.restype = ctypes.c_int
+            lib.oracle_decode.argtypes = [ctypes.POINTER(_DecodeArgs), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+            lib.oracle_decode.restype = ctypes.c_int
+            lib.oracle_lse_combine.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                               ctypes.c_void_p, ctypes.c_void_p]
+            lib.oracle_lse_combine.restype = None
+            lib.oracle_block_mask.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] + [ctypes.c_int] * 4 + \
+                [ctypes.c_void_p] * 5
+            lib.oracle_block_mask.restype = ctypes.c_int
+            lib.oracle_count_pairs.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] + [ctypes.c_int] * 2
+            lib.oracle_count_pairs.restype = ctypes.c_int64
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data
+
+
+def default_threads() -> int:
+    return os.cpu_count() or 1
+
+
+def attn(q, k, v, *, scale: Optional[float] = None, mask: int = MASK_NONE, window=(-1, -1), q_offset: int = 0,
+         doc_id=None, mod: int = MOD_NONE, softcap: float = 0.0, alibi=None, rows=None, kv_range=None,
+         nthreads: Optional[int] = None):
+    """Exact attention forward in fp64.
+
+    q: uint16 bf16 bits [B, Sq, Hq, D]; k, v: [B, Skv, Hkv, D] (any strides,
+    last dim contiguous). rows: optional int array [n, 3] of (b, h, i).
+    Returns (O, LSE): O float64 [B, Sq, Hq, D] and LSE [B, Hq, Sq] for all rows,
+    or O [n, D] and LSE [n] for the given rows.
+    """
+    lib = _load()
+    for t in (q, k, v):
+        assert t.dtype == np.uint16 and t.ndim == 4 and t.strides[3] == 2
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    a = _AttnArgs()
+    a.q, a.k, a.v = q.ctypes.data, k.ctypes.data, v.ctypes.data
+    a.q_sb, a.q_ss, a.q_sh = (s // 2 for s in q.strides[:3])
+    a.k_sb, a.k_ss, a.k_sh = (s // 2 for s in k.strides[:3])
+    a.v_sb, a.v_ss, a.v_sh = (s // 2 for s in v.strides[:3])
+    a.B, a.Hq, a.Hkv, a.Sq, a.Skv, a.D = B, Hq, Hkv, Sq, Skv, D
+    a.scale = (1.0 / np.sqrt(D)) if scale is None else float(scale)
+    a.mask, a.window_left, a.window_right, a.q_offset = mask, int(window[0]), int(window[1]), q_offset
+    doc = None if doc_id is None else np.ascontiguousarray(doc_id, dtype=np.int32)
+    a.doc_id = _ptr(doc)
+    a.mod, a.softcap = mod, float(softcap)
+    al = None
+    if alibi is not None:
+        al = np.ascontiguousarray(alibi, dtype=np.float32)
+        a.alibi_bstride = Hq if al.ndim == 2 else 0
+    a.alibi = _ptr(al)
+    a.kv_begin, a.kv_end = (0, Skv) if kv_range is None else (int(kv_range[0]), int(kv_range[1]))
+    nt = default_threads() if nthreads is None else nthreads
+    if rows is None:
+        n = B * Hq * Sq
+        o = np.empty((n, D), dtype=np.float64)
+        lse = np.empty(n, dtype=np.float64)
+        rc = lib.oracle_attn(ctypes.byref(a), None, n, o.ctypes.data, lse.ctypes.data, nt)
+        if rc != 0:
+            raise ValueError("oracle_attn: bad arguments")
+        return o.reshape(B, Hq, Sq, D).transpose(0, 2, 1, 3).copy(), lse.reshape(B, Hq, Sq)
+    r = np.ascontiguousarray(rows, dtype=np.int32).reshape(-1, 3)
+    n = r.shape[0]
+    o = np.empty((n, D), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64)
+    rc = lib.oracle_attn(ctypes.byref(a), r.ctypes.data, n, o.ctypes.data, lse.ctypes.data, nt)
+    if rc != 0:
+        raise ValueError("oracle_attn: bad arguments")
+    return o, lse
+
+
+def decode(q, k_cache, v_cache, block_table, cache_seqlens, *, scale: Optional[float] = None, mod: int = MOD_NONE,
+           softcap: float = 0.0, alibi=None, nthreads: Optional[int] = None):
+    """Single-query attention over a paged KV cache, fp64.
+
+    q: [B, 1, Hq, D] or [B, Hq, D] bf16 bits; k_cache/v_cache: [num_pages,
+    page_size, Hkv, D]; block_table int32 [B, max_pages]; cache_seqlens int32 [B].
+    Returns O float64 [B, Hq, D], LSE [B, Hq].
+    """
+    lib = _load()
+    if q.ndim == 4:
+        q = q[:, 0]
+    B, Hq, D = q.shape
+    P, page, Hkv, _ = k_cache.shape
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(cache_seqlens, dtype=np.int32)
+    a = _DecodeArgs()
+    a.q = q.ctypes.data
+    a.q_sb, a.q_sh = q.strides[0] // 2, q.strides[1] // 2
+    assert k_cache.strides == v_cache.strides
+    a.k_cache, a.v_cache = k_cache.ctypes.data, v_cache.ctypes.data
+    a.c_sp, a.c_ss, a.c_sh = (s // 2 for s in k_cache.strides[:3])
+    a.block_table, a.bt_stride, a.seqlens = bt.ctypes.data, bt.shape[1], sl.ctypes.data
+    a.B, a.Hq, a.Hkv, a.D, a.page_size, a.num_pages = B, Hq, Hkv, D, page, P
+    a.scale = (1.0 / np.sqrt(D)) if scale is None else float(scale)
+    a.mod, a.softcap = mod, float(softcap)
+    al = None
+    if alibi is not None:
+        al = np.ascontiguousarray(alibi, dtype=np.float32)
+        a.alibi_bstride = Hq if al.ndim == 2 else 0
+    a.alibi = _ptr(al)
+    o = np.empty((B, Hq, D), dtype=np.float64)
+    lse = np.empty((B, Hq), dtype=np.float64)
+    rc = lib.oracle_decode(ctypes.byref(a), o.ctypes.data, lse.ctypes.data,
+                           default_threads() if nthreads is None else nthreads)
+    if rc != 0:
+        raise ValueError("oracle_decode: bad arguments or page id out of range")
+    return o, lse
+
+
+def lse_combine(lse_parts, o_parts):
+    """Combine partial (LSE_i, O_i) over disjoint key sets. lse_parts [n], o_parts [n, D]."""
+    lib = _load()
+    lp = np.ascontiguousarray(lse_parts, dtype=np.float64)
+    op = np.ascontiguousarray(o_parts, dtype=np.float64)
+    D = op.shape[1]
+    o = np.empty(D, dtype=np.float64)
+    lse = np.empty(1, dtype=np.float64)
+    lib.oracle_lse_combine(lp.shape[0], lp.ctypes.data, op.ctypes.data, D, o.ctypes.data, lse.ctypes.data)
+    return o, float(lse[0])
+
+
+def block_mask(mask: int, Sq: int, Skv: int, blk_q: int = 128, blk_kv: int = 128, window=(-1, -1),
+               q_offset: int = 0, doc_id=None) -> dict:
+    """Brute-force tile classification: dict(cls, part_cnt, part_idx, full_cnt, full_idx).
+
+    The *_idx arrays are [nQ, nK] with entries past the count set to -1.
+    """
+    lib = _load()
+    nQ, nK = -(-Sq // blk_q), -(-Skv // blk_kv)
+    cls = np.zeros((nQ, nK), dtype=np.uint8)
+    pc = np.zeros(nQ, dtype=np.int32)
+    fc = np.zeros(nQ, dtype=np.int32)
+    pi = np.full((nQ, nK), -1, dtype=np.int32)
+    fi = np.full((nQ, nK), -1, dtype=np.int32)
+    doc = None if doc_id is None else np.ascontiguousarray(doc_id, dtype=np.int32)
+    rc = lib.oracle_block_mask(mask, int(window[0]), int(window[1]), q_offset, _ptr(doc), Sq, Skv, blk_q, blk_kv,
+                               cls.ctypes.data, pc.ctypes.data, pi.ctypes.data, fc.ctypes.data, fi.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_block_mask: bad arguments")
+    return dict(cls=cls, part_cnt=pc, part_idx=pi, full_cnt=fc, full_idx=fi)
+
+
+def count_pairs(mask: int, Sq: int, Skv: int, window=(-1, -1), q_offset: int = 0, doc_id=None) -> int:
+    """Allowed (q, kv) pairs of one (batch, head) under the mask."""
+    lib = _load()
+    doc = None if doc_id is None else np.ascontiguousarray(doc_id, dtype=np.int32)
+    return int(lib.oracle_count_pairs(mask, int(window[0]), int(window[1]), q_offset, _ptr(doc), Sq, Skv))
