@@ -1,0 +1,264 @@
+"""Exact attention forward on B200 (sm_100a): Python binding of libattn.
+
+Every function here only marshals arguments into the C ABI of
+include/attn.h (pointers, sizes, strides, the current CUDA stream). All of
+the computation runs in the library's CUDA kernels; PyTorch supplies device
+memory and streams. There is no CPU or PyTorch fallback: if libattn.so is
+missing or a call fails, an exception is raised.
+
+Entry points (same names as the C ABI):
+  attn_fwd(q, k, v, ...)            prefill / full-sequence forward -> (O, LSE)
+  attn_decode(q, k_cache, ...)      split-KV paged decode          -> (O, LSE)
+  attn_build_block_mask(...)        FlexAttention-style block mask -> BlockMask
+  attn_lse_combine(o_parts, ...)    merge split partial results    -> (O, LSE)
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+from . import _lib
+from ._lib import (ATTN_DEV_BAD_PAGE, ATTN_DEV_TIMEOUT, MASK_CAUSAL, MASK_DOCUMENT, MASK_NONE, MASK_WINDOW,
+                   MOD_ALIBI, MOD_NONE, MOD_SOFTCAP, AttnError)
+
+__all__ = ["attn_fwd", "attn_decode", "attn_build_block_mask", "attn_lse_combine", "BlockMask", "AttnError",
+           "load_library", "ATTN_DEV_TIMEOUT", "ATTN_DEV_BAD_PAGE"]
+
+
+def load_library():
+    return _lib.load()
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(device) -> int:
+    torch = _torch()
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check_bf16(name, t, ndim):
+    torch = _torch()
+    if t.dtype != torch.bfloat16:
+        raise TypeError("%s must be bfloat16, got %s" % (name, t.dtype))
+    if t.dim() != ndim:
+        raise ValueError("%s must have %d dims, got %d" % (name, ndim, t.dim()))
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.stride(-1) != 1:
+        raise ValueError("%s: the head dimension must be contiguous" % name)
+
+
+class BlockMask:
+    """Tile-level mask (FlexAttention BlockMask equivalent) in one device buffer.
+
+    cls[q_tile, kv_tile] is 0 (empty), 1 (partial) or 2 (full); part_idx /
+    full_idx list the partial / full kv tiles of each q tile in ascending order,
+    the first part_cnt / full_cnt entries of each row being valid.
+    """
+
+    def __init__(self, Sq: int, Skv: int, blk_q: int, blk_kv: int, device):
+        torch = _torch()
+        lib = _lib.load()
+        nbytes = lib.attn_block_mask_bytes(Sq, Skv, blk_q, blk_kv)
+        if nbytes == 0:
+            raise ValueError("invalid block mask sizes")
+        self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.c = _lib.BlockMaskC()
+        _lib.check(lib.attn_block_mask_layout(self.buffer.data_ptr(), nbytes, Sq, Skv, blk_q, blk_kv,
+                                              ctypes.byref(self.c)), "attn_block_mask_layout")
+        self.Sq, self.Skv, self.blk_q, self.blk_kv = Sq, Skv, blk_q, blk_kv
+        self.shape = (self.c.n_q_tiles, self.c.n_kv_tiles)
+
+    def _view(self, addr, dtype, shape):
+        torch = _torch()
+        off = addr - self.buffer.data_ptr()
+        n = 1
+        for s in shape:
+            n *= s
+        esz = torch.empty((), dtype=dtype).element_size()
+        return self.buffer[off:off + n * esz].view(dtype).view(*shape)
+
+    @property
+    def cls(self):
+        return self._view(self.c.cls, _torch().uint8, self.shape)
+
+    @property
+    def part_cnt(self):
+        return self._view(self.c.part_cnt, _torch().int32, (self.shape[0],))
+
+    @property
+    def full_cnt(self):
+        return self._view(self.c.full_cnt, _torch().int32, (self.shape[0],))
+
+    @property
+    def part_idx(self):
+        return self._view(self.c.part_idx, _torch().int32, self.shape)
+
+    @property
+    def full_idx(self):
+        return self._view(self.c.full_idx, _torch().int32, self.shape)
+
+
+def _mask_spec(causal: bool, window, q_offset: int, doc_id) -> Tuple[_lib.MaskSpec, int]:
+    spec = _lib.MaskSpec()
+    wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    if doc_id is not None:
+        kind = MASK_DOCUMENT
+    elif causal:
+        kind = MASK_CAUSAL
+    elif (wl, wr) != (-1, -1):
+        kind = MASK_WINDOW
+    else:
+        kind = MASK_NONE
+    spec.kind, spec.window_left, spec.window_right, spec.q_offset = kind, wl, wr, int(q_offset)
+    spec.doc_id = _ptr(doc_id)
+    return spec, kind
+
+
+def attn_build_block_mask(Sq: int, Skv: int, *, causal: bool = False, window=None, q_offset: int = 0,
+                          doc_id=None, blk_q: int = 128, blk_kv: int = 128, device=None, stream=None) -> BlockMask:
+    """Classify every (q-tile, kv-tile) of the mask on the device."""
+    torch = _torch()
+    if doc_id is not None:
+        if doc_id.dtype != torch.int32 or not doc_id.is_cuda or not doc_id.is_contiguous():
+            raise ValueError("doc_id must be a contiguous int32 CUDA tensor")
+        device = doc_id.device
+    device = device if device is not None else torch.device("cuda")
+    bm = BlockMask(Sq, Skv, blk_q, blk_kv, device)
+    spec, _ = _mask_spec(causal, window, q_offset, doc_id)
+    h = _stream_handle(device) if stream is None else stream
+    _lib.check(_lib.load().attn_build_block_mask(ctypes.byref(spec), ctypes.byref(bm.c), h),
+               "attn_build_block_mask")
+    bm._doc_id = doc_id
+    return bm
+
+
+def _mod_args(softcap, alibi_slopes, Hq):
+    torch = _torch()
+    if softcap is not None and alibi_slopes is not None:
+        raise ValueError("choose one score mod: softcap or alibi_slopes")
+    if softcap is not None:
+        return MOD_SOFTCAP, float(softcap), None, 0
+    if alibi_slopes is not None:
+        if alibi_slopes.dtype != torch.float32 or not alibi_slopes.is_cuda or not alibi_slopes.is_contiguous():
+            raise ValueError("alibi_slopes must be a contiguous fp32 CUDA tensor")
+        stride = 0 if alibi_slopes.dim() == 1 else Hq
+        return MOD_ALIBI, 0.0, alibi_slopes.data_ptr(), stride
+    return MOD_NONE, 0.0, None, 0
+
+
+def attn_fwd(q, k, v, *, scale: Optional[float] = None, causal: bool = False, window=None, q_offset: int = 0,
+             doc_id=None, block_mask: Optional[BlockMask] = None, softcap: Optional[float] = None,
+             alibi_slopes=None, out=None, lse=None, status=None, with_lse: bool = True, stream=None):
+    """Exact attention forward. q [B, Sq, Hq, D], k/v [B, Skv, Hkv, D] bf16 (any
+    strides with a contiguous last dim, e.g. BHSD views). Returns (O, LSE):
+    O bf16 [B, Sq, Hq, D] and LSE fp32 [B, Hq, Sq] (natural log)."""
+    torch = _torch()
+    _check_bf16("q", q, 4)
+    _check_bf16("k", k, 4)
+    _check_bf16("v", v, 4)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty((B, Sq, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and with_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    p = _lib.FwdParams()
+    p.q, p.k, p.v, p.o = q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr()
+    p.lse = _ptr(lse)
+    p.q_stride = _lib.c_i64x3(*q.stride()[:3])
+    p.k_stride = _lib.c_i64x3(*k.stride()[:3])
+    p.v_stride = _lib.c_i64x3(*v.stride()[:3])
+    p.o_stride = _lib.c_i64x3(*out.stride()[:3])
+    p.B, p.Hq, p.Hkv, p.Sq, p.Skv, p.D = B, Hq, Hkv, Sq, Skv, D
+    p.scale = 0.0 if scale is None else float(scale)
+    spec, kind = _mask_spec(causal, window, q_offset, doc_id)
+    p.mask = spec
+    if kind == MASK_DOCUMENT and block_mask is None:
+        block_mask = attn_build_block_mask(Sq, Skv, doc_id=doc_id, stream=stream)
+    p.block_mask = ctypes.pointer(block_mask.c) if block_mask is not None else None
+    p.mod, p.softcap, p.alibi_slopes, p.alibi_batch_stride = _mod_args(softcap, alibi_slopes, Hq)
+    p.status = _ptr(status)
+    h = _stream_handle(q.device) if stream is None else stream
+    _lib.check(_lib.load().attn_fwd(ctypes.byref(p), h), "attn_fwd")
+    return out, lse
+
+
+def attn_decode(q, k_cache, v_cache, block_table, cache_seqlens, *, max_seqlen: Optional[int] = None,
+                scale: Optional[float] = None, softcap: Optional[float] = None, alibi_slopes=None,
+                num_splits: int = 0, out=None, lse=None, workspace=None, status=None, with_lse: bool = True,
+                stream=None):
+    """Split-KV decode over a paged cache. q [B, Hq, D] (or [B, 1, Hq, D]);
+    k_cache/v_cache [num_pages, page_size, Hkv, D]; block_table int32
+    [B, max_pages]; cache_seqlens int32 [B]. Returns (O [B, Hq, D], LSE [B, Hq])."""
+    torch = _torch()
+    if q.dim() == 4:
+        q = q[:, 0]
+    _check_bf16("q", q, 3)
+    _check_bf16("k_cache", k_cache, 4)
+    _check_bf16("v_cache", v_cache, 4)
+    if k_cache.stride() != v_cache.stride():
+        raise ValueError("k_cache and v_cache must share strides")
+    for name, t in (("block_table", block_table), ("cache_seqlens", cache_seqlens)):
+        if t.dtype != torch.int32 or not t.is_cuda:
+            raise ValueError("%s must be an int32 CUDA tensor" % name)
+    if block_table.stride(1) != 1 or not cache_seqlens.is_contiguous():
+        raise ValueError("block_table rows and cache_seqlens must be contiguous")
+    B, Hq, D = q.shape
+    P, page, Hkv, _ = k_cache.shape
+    if max_seqlen is None:
+        max_seqlen = block_table.shape[1] * page
+    lib = _lib.load()
+    splits = lib.attn_decode_num_splits(B, Hq, Hkv, int(max_seqlen), int(num_splits))
+    need = lib.attn_decode_workspace_bytes(B, Hq, D, splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and with_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    p = _lib.DecodeParams()
+    p.q = q.data_ptr()
+    p.q_stride = _lib.c_i64x2(q.stride(0), q.stride(1))
+    p.k_cache, p.v_cache = k_cache.data_ptr(), v_cache.data_ptr()
+    p.cache_stride = _lib.c_i64x3(*k_cache.stride()[:3])
+    p.block_table, p.block_table_stride = block_table.data_ptr(), block_table.stride(0)
+    p.cache_seqlens = cache_seqlens.data_ptr()
+    p.B, p.Hq, p.Hkv, p.D, p.page_size, p.num_pages = B, Hq, Hkv, D, page, P
+    p.max_seqlen = int(max_seqlen)
+    p.scale = 0.0 if scale is None else float(scale)
+    p.mod, p.softcap, p.alibi_slopes, p.alibi_batch_stride = _mod_args(softcap, alibi_slopes, Hq)
+    p.num_splits = int(num_splits)
+    p.o = out.data_ptr()
+    p.o_stride = _lib.c_i64x2(out.stride(0), out.stride(1))
+    p.lse = _ptr(lse)
+    p.status = _ptr(status)
+    h = _stream_handle(q.device) if stream is None else stream
+    _lib.check(lib.attn_decode(ctypes.byref(p), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                               h), "attn_decode")
+    return out, lse
+
+
+def attn_lse_combine(o_parts, lse_parts, *, out=None, lse=None, stream=None):
+    """Merge split partials: o_parts fp32 [rows, n, D], lse_parts fp32 [rows, n]."""
+    torch = _torch()
+    rows, n, D = o_parts.shape
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
+        raise TypeError("partials must be fp32")
+    if not (o_parts.is_contiguous() and lse_parts.is_contiguous()):
+        raise ValueError("partials must be contiguous")
+    if out is None:
+        out = torch.empty((rows, D), dtype=torch.bfloat16, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((rows,), dtype=torch.float32, device=o_parts.device)
+    h = _stream_handle(o_parts.device) if stream is None else stream
+    _lib.check(_lib.load().attn_lse_combine(o_parts.data_ptr(), lse_parts.data_ptr(), rows, n, D, out.data_ptr(),
+                                            out.stride(0), _ptr(lse), h), "attn_lse_combine")
+    return out, lse

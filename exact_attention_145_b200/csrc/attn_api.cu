@@ -1,0 +1,434 @@
+// attn_api.cu - the C ABI declared in include/attn.h: host-side argument
+// checks, TMA tensor-map encoding, work decomposition and kernel launches.
+// Nothing here allocates device memory or synchronises a stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "aux_kernels.cuh"
+#include "fwd_kernel.cuh"
+
+using namespace attn_kernels;
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A bf16 tensor map over (dims[0] contiguous, dims[1..r-1] with element
+// strides), box = {64, box_rows, 1, ...}, 128-byte swizzle.
+attn_status make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const int64_t* strides_el,
+                     uint32_t box_rows, int box_rows_dim) {
+  auto enc = encoder();
+  if (!enc) return ATTN_ERR_CUDA;
+  cuuint64_t gdim[5];
+  cuuint64_t gstride[4];
+  cuuint32_t box[5];
+  cuuint32_t es[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    box[i] = 1;
+    es[i] = 1;
+    if (dims[i] == 0 || dims[i] > (1ull << 32)) return ATTN_ERR_UNSUPPORTED;
+  }
+  box[0] = 64;
+  box[box_rows_dim] = box_rows;
+  for (int i = 1; i < rank; ++i) {
+    const int64_t b = strides_el[i - 1] * 2;
+    if (b <= 0 || (b % 16) != 0 || b >= (1ll << 40)) return ATTN_ERR_UNSUPPORTED;
+    gstride[i - 1] = static_cast<cuuint64_t>(b);
+  }
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gdim, gstride, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
+}
+
+// The dynamic shared-memory opt-in is per device; remember which devices
+// have it for each kernel instantiation.
+template <int D, bool DECODE>
+attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdArgs& a,
+                       int grid, cudaStream_t stream) {
+  using L = Layout<D, DECODE>;
+  static std::mutex mu;
+  static uint64_t ready_mask = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!(ready_mask & (1ull << dev))) {
+      if (cudaFuncSetAttribute(attn_fwd_kernel<D, DECODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               L::kSmemBytes) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+      ready_mask |= 1ull << dev;
+    }
+  }
+  attn_fwd_kernel<D, DECODE><<<grid, kThreads, L::kSmemBytes, stream>>>(mq, mk, mv, a);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+bool strides_ok(const int64_t* s, int n) {
+  for (int i = 0; i < n; ++i)
+    if (s[i] < 0 || (s[i] % 8) != 0) return false;
+  return true;
+}
+
+attn_status check_mods(attn_mod_kind mod, float softcap, const float* alibi, int alibi_bstride, int Hq) {
+  if (mod == ATTN_MOD_SOFTCAP && !(softcap > 0.f && std::isfinite(softcap))) return ATTN_ERR_INVALID_ARG;
+  if (mod == ATTN_MOD_ALIBI && (alibi == nullptr || (alibi_bstride != 0 && alibi_bstride != Hq)))
+    return ATTN_ERR_INVALID_ARG;
+  if (mod != ATTN_MOD_NONE && mod != ATTN_MOD_SOFTCAP && mod != ATTN_MOD_ALIBI) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_str(attn_status s) {
+  switch (s) {
+    case ATTN_OK:
+      return "ok";
+    case ATTN_ERR_INVALID_ARG:
+      return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED:
+      return "unsupported configuration";
+    case ATTN_ERR_CUDA:
+      return "CUDA error";
+    case ATTN_ERR_WORKSPACE:
+      return "workspace too small";
+  }
+  return "unknown status";
+}
+
+size_t attn_block_mask_bytes(int Sq, int Skv, int blk_q, int blk_kv) {
+  if (Sq <= 0 || Skv <= 0 || blk_q <= 0 || blk_kv <= 0) return 0;
+  const size_t nQ = (Sq + blk_q - 1) / blk_q, nK = (Skv + blk_kv - 1) / blk_kv;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  return up(nQ * nK) + 2 * up(nQ * 4) + 2 * up(nQ * nK * 4);
+}
+
+attn_status attn_block_mask_layout(void* buf, size_t buf_bytes, int Sq, int Skv, int blk_q, int blk_kv,
+                                   attn_block_mask* out) {
+  if (!out || !buf || !aligned16(buf)) return ATTN_ERR_INVALID_ARG;
+  const size_t need = attn_block_mask_bytes(Sq, Skv, blk_q, blk_kv);
+  if (need == 0) return ATTN_ERR_INVALID_ARG;
+  if (buf_bytes < need) return ATTN_ERR_WORKSPACE;
+  const size_t nQ = (Sq + blk_q - 1) / blk_q, nK = (Skv + blk_kv - 1) / blk_kv;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  uint8_t* p = static_cast<uint8_t*>(buf);
+  out->Sq = Sq;
+  out->Skv = Skv;
+  out->blk_q = blk_q;
+  out->blk_kv = blk_kv;
+  out->n_q_tiles = static_cast<int>(nQ);
+  out->n_kv_tiles = static_cast<int>(nK);
+  out->cls = p;
+  p += up(nQ * nK);
+  out->part_cnt = reinterpret_cast<int32_t*>(p);
+  p += up(nQ * 4);
+  out->full_cnt = reinterpret_cast<int32_t*>(p);
+  p += up(nQ * 4);
+  out->part_idx = reinterpret_cast<int32_t*>(p);
+  p += up(nQ * nK * 4);
+  out->full_idx = reinterpret_cast<int32_t*>(p);
+  return ATTN_OK;
+}
+
+attn_status attn_build_block_mask(const attn_mask_spec* spec, const attn_block_mask* out, void* stream) {
+  if (!spec || !out) return ATTN_ERR_INVALID_ARG;
+  if (out->Sq <= 0 || out->Skv <= 0 || out->blk_q <= 0 || out->blk_kv <= 0) return ATTN_ERR_INVALID_ARG;
+  if (out->blk_q % 16 || out->blk_kv % 16 || out->blk_q > 1024 || out->blk_kv > 1024) return ATTN_ERR_UNSUPPORTED;
+  if (out->n_q_tiles != (out->Sq + out->blk_q - 1) / out->blk_q ||
+      out->n_kv_tiles != (out->Skv + out->blk_kv - 1) / out->blk_kv)
+    return ATTN_ERR_INVALID_ARG;
+  if (!out->cls || !out->part_cnt || !out->part_idx || !out->full_cnt || !out->full_idx) return ATTN_ERR_INVALID_ARG;
+  if (spec->kind < ATTN_MASK_NONE || spec->kind > ATTN_MASK_DOCUMENT) return ATTN_ERR_INVALID_ARG;
+  if (spec->kind == ATTN_MASK_DOCUMENT && (!spec->doc_id || out->Sq != out->Skv || spec->q_offset != 0))
+    return ATTN_ERR_INVALID_ARG;
+  MaskArgs a;
+  a.kind = spec->kind;
+  a.wl = spec->kind == ATTN_MASK_CAUSAL ? -1 : spec->window_left;
+  a.wr = spec->kind == ATTN_MASK_CAUSAL ? 0 : spec->window_right;
+  a.q_offset = spec->kind == ATTN_MASK_NONE ? 0 : spec->q_offset;
+  a.doc_id = spec->doc_id;
+  a.Sq = out->Sq;
+  a.Skv = out->Skv;
+  a.blk_q = out->blk_q;
+  a.blk_kv = out->blk_kv;
+  a.nQ = out->n_q_tiles;
+  a.nK = out->n_kv_tiles;
+  a.cls = out->cls;
+  a.part_cnt = out->part_cnt;
+  a.part_idx = out->part_idx;
+  a.full_cnt = out->full_cnt;
+  a.full_idx = out->full_idx;
+  const size_t smem = (size_t)(a.blk_q + a.blk_kv) * sizeof(int);
+  build_block_mask_kernel<<<a.nQ, kMaskThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
+  if (!p) return ATTN_ERR_INVALID_ARG;
+  if (p->B < 0 || p->Sq < 0 || p->Skv < 0 || p->Hq <= 0 || p->Hkv <= 0) return ATTN_ERR_INVALID_ARG;
+  if (p->Hq % p->Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (p->D != 64 && p->D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (p->B == 0 || p->Sq == 0) return ATTN_OK;
+  if (!p->q || !p->o || (p->Skv > 0 && (!p->k || !p->v))) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(p->q) || !aligned16(p->o) || (p->k && !aligned16(p->k)) || (p->v && !aligned16(p->v)))
+    return ATTN_ERR_UNSUPPORTED;
+  if (!strides_ok(p->q_stride, 3) || !strides_ok(p->k_stride, 3) || !strides_ok(p->v_stride, 3) ||
+      !strides_ok(p->o_stride, 3))
+    return ATTN_ERR_UNSUPPORTED;
+  if (p->mask.kind < ATTN_MASK_NONE || p->mask.kind > ATTN_MASK_DOCUMENT) return ATTN_ERR_INVALID_ARG;
+  if (attn_status st = check_mods(p->mod, p->softcap, p->alibi_slopes, p->alibi_batch_stride, p->Hq)) return st;
+  const int nQ = (p->Sq + kRows - 1) / kRows;
+  const int nK = (p->Skv + kKeys - 1) / kKeys;
+  if (p->mask.kind == ATTN_MASK_DOCUMENT) {
+    if (!p->mask.doc_id || p->Sq != p->Skv || p->mask.q_offset != 0 || !p->block_mask) return ATTN_ERR_INVALID_ARG;
+  }
+  if (p->block_mask) {
+    const attn_block_mask* bm = p->block_mask;
+    if (bm->blk_q != kRows || bm->blk_kv != kKeys || bm->Sq != p->Sq || bm->Skv != p->Skv || !bm->cls ||
+        bm->n_q_tiles != nQ || bm->n_kv_tiles != nK)
+      return ATTN_ERR_INVALID_ARG;
+  }
+
+  FwdArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.Sq = p->Sq;
+  a.Skv = p->Skv;
+  a.g = p->Hq / p->Hkv;
+  a.scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
+  a.scale_log2 = a.scale * kLog2e;
+  a.mask = p->mask.kind;
+  switch (p->mask.kind) {
+    case ATTN_MASK_NONE:
+      a.wl = a.wr = -1;
+      a.q_offset = 0;
+      break;
+    case ATTN_MASK_CAUSAL:
+      a.wl = -1;
+      a.wr = 0;
+      a.q_offset = p->mask.q_offset;
+      break;
+    case ATTN_MASK_WINDOW:
+      a.wl = p->mask.window_left < 0 ? -1 : p->mask.window_left;
+      a.wr = p->mask.window_right < 0 ? -1 : p->mask.window_right;
+      a.q_offset = p->mask.q_offset;
+      break;
+    default:
+      a.wl = -1;
+      a.wr = 0;
+      a.q_offset = 0;
+  }
+  a.doc_id = p->mask.doc_id;
+  a.bm_cls = p->block_mask ? p->block_mask->cls : nullptr;
+  a.nQ = nQ;
+  a.nK = nK;
+  a.mod = p->mod;
+  a.softcap = p->softcap;
+  a.alibi = p->alibi_slopes;
+  a.alibi_bstride = p->alibi_batch_stride;
+  a.o = static_cast<__nv_bfloat16*>(p->o);
+  a.o_sb = p->o_stride[0];
+  a.o_ss = p->o_stride[1];
+  a.o_sh = p->o_stride[2];
+  a.lse = p->lse;
+  a.status = p->status;
+  a.pair_heads = (a.g % 2 == 0) ? 1 : 0;
+  a.n_row_units = a.pair_heads ? nQ : (nQ + 1) / 2;
+
+  CUtensorMap mq, mk, mv;
+  const uint64_t dq[4] = {(uint64_t)p->D, (uint64_t)p->Sq, (uint64_t)p->Hq, (uint64_t)p->B};
+  const int64_t sq[3] = {p->q_stride[1], p->q_stride[2], p->q_stride[0]};
+  // Skv == 0: every row is fully masked; the maps are never read (no tile is visited).
+  const uint64_t dk[4] = {(uint64_t)p->D, (uint64_t)(p->Skv > 0 ? p->Skv : 1), (uint64_t)p->Hkv, (uint64_t)p->B};
+  const int64_t sk[3] = {p->k_stride[1], p->k_stride[2], p->k_stride[0]};
+  const int64_t sv[3] = {p->v_stride[1], p->v_stride[2], p->v_stride[0]};
+  // Degenerate strides of size-1 dims still have to pass the encoder's checks.
+  int64_t sq2[3], sk2[3], sv2[3];
+  for (int i = 0; i < 3; ++i) {
+    sq2[i] = sq[i] > 0 ? sq[i] : 8;
+    sk2[i] = sk[i] > 0 ? sk[i] : 8;
+    sv2[i] = sv[i] > 0 ? sv[i] : 8;
+  }
+  if (attn_status st = make_map(&mq, p->q, 4, dq, sq2, kRows, 1)) return st;
+  // With Skv == 0 nothing is read from K / V; the unused maps point at Q.
+  if (attn_status st = make_map(&mk, p->Skv > 0 ? p->k : p->q, 4, dk, sk2, kKeys, 1)) return st;
+  if (attn_status st = make_map(&mv, p->Skv > 0 ? p->v : p->q, 4, dk, sv2, kKeys, 1)) return st;
+
+  const int HU = a.pair_heads ? a.Hq / 2 : a.Hq;
+  const long grid = (long)a.B * HU * a.n_row_units;
+  if (grid <= 0 || grid > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return p->D == 128 ? launch_fwd<128, false>(mq, mk, mv, a, (int)grid, s)
+                     : launch_fwd<64, false>(mq, mk, mv, a, (int)grid, s);
+}
+
+int attn_decode_num_splits(int B, int Hq, int Hkv, int max_seqlen, int num_splits) {
+  if (B <= 0 || Hkv <= 0 || Hq <= 0 || max_seqlen <= 0) return 1;
+  const int tiles = (max_seqlen + kKeys - 1) / kKeys;
+  if (num_splits > 0) return num_splits < tiles ? num_splits : tiles;
+  // Pick the split count that minimises (waves of CTAs) x (tiles per split),
+  // favouring fewer splits on ties (less partial traffic).
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms <= 0) sms = 148;
+  const long units = (long)B * Hkv;
+  int best = 1;
+  long best_cost = -1;
+  for (int n = 1; n <= tiles && n <= 256; ++n) {
+    const long waves = (units * n + sms - 1) / sms;
+    const long per = (tiles + n - 1) / n;
+    const long cost = waves * (per + 2);  // +2 tiles' worth of fixed per-CTA cost
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = n;
+    }
+  }
+  return best;
+}
+
+size_t attn_decode_workspace_bytes(int B, int Hq, int D, int num_splits) {
+  if (B <= 0 || Hq <= 0 || D <= 0 || num_splits <= 0) return 0;
+  const size_t rows = (size_t)B * Hq * num_splits;
+  const size_t o_bytes = (rows * D * sizeof(float) + 255) & ~size_t(255);
+  return o_bytes + rows * sizeof(float);
+}
+
+static attn_status launch_combine(const CombineArgs& c, int D, cudaStream_t s) {
+  const int warps = 8;
+  const int grid = (c.rows + warps - 1) / warps;
+  if (D == 128)
+    lse_combine_kernel<128><<<grid, warps * 32, 0, s>>>(c);
+  else
+    lse_combine_kernel<64><<<grid, warps * 32, 0, s>>>(c);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status attn_decode(const attn_decode_params* p, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!p) return ATTN_ERR_INVALID_ARG;
+  if (p->B < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->page_size <= 0 || p->num_pages <= 0) return ATTN_ERR_INVALID_ARG;
+  if (p->Hq % p->Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (p->D != 64 && p->D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (p->Hq / p->Hkv > kRows) return ATTN_ERR_UNSUPPORTED;
+  if (p->page_size % 16 != 0 || (p->page_size < kKeys && kKeys % p->page_size != 0) ||
+      (p->page_size > kKeys && p->page_size % kKeys != 0))
+    return ATTN_ERR_UNSUPPORTED;
+  if (p->B == 0) return ATTN_OK;
+  if (!p->q || !p->k_cache || !p->v_cache || !p->block_table || !p->cache_seqlens || !p->o)
+    return ATTN_ERR_INVALID_ARG;
+  if (p->max_seqlen <= 0 || p->block_table_stride <= 0) return ATTN_ERR_INVALID_ARG;
+  if ((long)p->block_table_stride * p->page_size < p->max_seqlen) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->o))
+    return ATTN_ERR_UNSUPPORTED;
+  if (!strides_ok(p->q_stride, 2) || !strides_ok(p->cache_stride, 3) || !strides_ok(p->o_stride, 2))
+    return ATTN_ERR_UNSUPPORTED;
+  if (attn_status st = check_mods(p->mod, p->softcap, p->alibi_slopes, p->alibi_batch_stride, p->Hq)) return st;
+  const int splits = attn_decode_num_splits(p->B, p->Hq, p->Hkv, p->max_seqlen, p->num_splits);
+  const size_t need = attn_decode_workspace_bytes(p->B, p->Hq, p->D, splits);
+  if (!workspace || !aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+
+  FwdArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.g = p->Hq / p->Hkv;
+  a.scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
+  a.scale_log2 = a.scale * kLog2e;
+  a.mask = MASK_NONE;
+  a.wl = a.wr = -1;
+  a.mod = p->mod;
+  a.softcap = p->softcap;
+  a.alibi = p->alibi_slopes;
+  a.alibi_bstride = p->alibi_batch_stride;
+  a.status = p->status;
+  a.block_table = p->block_table;
+  a.bt_stride = p->block_table_stride;
+  a.seqlens = p->cache_seqlens;
+  a.page_size = p->page_size;
+  a.num_pages = p->num_pages;
+  a.box_rows = p->page_size < kKeys ? p->page_size : kKeys;
+  const int tiles = (p->max_seqlen + kKeys - 1) / kKeys;
+  a.n_splits = splits;
+  a.tiles_per_split = (tiles + splits - 1) / splits;
+  const size_t rows = (size_t)p->B * p->Hq * splits;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((rows * p->D * 4 + 255) & ~size_t(255)));
+
+  CUtensorMap mq, mk, mv;
+  const uint64_t dq[3] = {(uint64_t)p->D, (uint64_t)p->Hq, (uint64_t)p->B};
+  const int64_t sq[2] = {p->q_stride[1] > 0 ? p->q_stride[1] : 8, p->q_stride[0] > 0 ? p->q_stride[0] : 8};
+  const uint64_t dc[4] = {(uint64_t)p->D, (uint64_t)p->Hkv, (uint64_t)p->page_size, (uint64_t)p->num_pages};
+  const int64_t sc[3] = {p->cache_stride[2] > 0 ? p->cache_stride[2] : 8, p->cache_stride[1],
+                         p->cache_stride[0]};
+  if (attn_status st = make_map(&mq, p->q, 3, dq, sq, kRows, 1)) return st;
+  if (attn_status st = make_map(&mk, p->k_cache, 4, dc, sc, (uint32_t)a.box_rows, 2)) return st;
+  if (attn_status st = make_map(&mv, p->v_cache, 4, dc, sc, (uint32_t)a.box_rows, 2)) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long grid = (long)p->B * p->Hkv * splits;
+  if (grid > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+  attn_status st = p->D == 128 ? launch_fwd<128, true>(mq, mk, mv, a, (int)grid, s)
+                               : launch_fwd<64, true>(mq, mk, mv, a, (int)grid, s);
+  if (st != ATTN_OK) return st;
+  CombineArgs c;
+  c.o_parts = a.part_o;
+  c.lse_parts = a.part_lse;
+  c.rows = p->B * p->Hq;
+  c.n = splits;
+  c.D = p->D;
+  c.rows_per_b = p->Hq;
+  c.o = static_cast<__nv_bfloat16*>(p->o);
+  c.o_sb = p->o_stride[0];
+  c.o_sh = p->o_stride[1];
+  c.lse = p->lse;
+  return launch_combine(c, p->D, s);
+}
+
+attn_status attn_lse_combine(const float* o_parts, const float* lse_parts, int rows, int n_splits, int D, void* o,
+                             int64_t o_row_stride, float* lse, void* stream) {
+  if (rows < 0 || n_splits <= 0 || (D != 64 && D != 128)) return rows < 0 || n_splits <= 0 ? ATTN_ERR_INVALID_ARG
+                                                                                          : ATTN_ERR_UNSUPPORTED;
+  if (rows == 0) return ATTN_OK;
+  if (!o_parts || !lse_parts || !o) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || (reinterpret_cast<uintptr_t>(o) & 7u) || o_row_stride < D || (o_row_stride % 4))
+    return ATTN_ERR_UNSUPPORTED;
+  CombineArgs c;
+  c.o_parts = o_parts;
+  c.lse_parts = lse_parts;
+  c.rows = rows;
+  c.n = n_splits;
+  c.D = D;
+  c.rows_per_b = rows;
+  c.o = static_cast<__nv_bfloat16*>(o);
+  c.o_sb = 0;
+  c.o_sh = o_row_stride;
+  c.lse = lse;
+  return launch_combine(c, D, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

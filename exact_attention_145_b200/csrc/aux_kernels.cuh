@@ -1,0 +1,147 @@
+// aux_kernels.cuh - CUDA-core kernels around the attention forward:
+//   * block-mask builder (FlexAttention create_block_mask equivalent)
+//   * LSE combine of split-KV partial results
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace attn_kernels {
+
+struct MaskArgs {
+  int kind, wl, wr, q_offset;
+  const int32_t* doc_id;
+  int Sq, Skv, blk_q, blk_kv, nQ, nK;
+  uint8_t* cls;
+  int32_t *part_cnt, *part_idx, *full_cnt, *full_idx;
+};
+
+__device__ __forceinline__ bool mask_allows(const MaskArgs& a, int i, int j, int doc_i, const int* doc_j_smem,
+                                            int jl) {
+  const long q_pos = (long)i + a.q_offset;
+  switch (a.kind) {
+    case 0:
+      return true;
+    case 1:
+      return (long)j <= q_pos;
+    case 2:
+      return (a.wl < 0 || q_pos - j <= a.wl) && (a.wr < 0 || (long)j - q_pos <= a.wr);
+    default:
+      return (long)j <= q_pos && doc_j_smem[jl] == doc_i;
+  }
+}
+
+// One CTA per q-tile. For every kv-tile the block evaluates the mask on all
+// in-range (q, kv) pairs of the tile, reduces "any allowed" and "all allowed"
+// with block-wide votes, and thread 0 appends the tile to the partial or full
+// list, so both lists come out in ascending kv order.
+constexpr int kMaskThreads = 256;
+
+__global__ void __launch_bounds__(kMaskThreads) build_block_mask_kernel(const MaskArgs a) {
+  extern __shared__ int doc_smem[];  // [blk_q] query doc ids, then [blk_kv] key doc ids
+  int* doc_q = doc_smem;
+  int* doc_k = doc_smem + a.blk_q;
+  const int qt = blockIdx.x;
+  const int q0 = qt * a.blk_q;
+  const int rows = min(a.blk_q, a.Sq - q0);
+  const bool is_doc = a.kind == 3;
+  if (is_doc)
+    for (int r = threadIdx.x; r < rows; r += blockDim.x) doc_q[r] = a.doc_id[q0 + r];
+  int np = 0, nf = 0;
+  for (int kt = 0; kt < a.nK; ++kt) {
+    const int k0 = kt * a.blk_kv;
+    const int cols = min(a.blk_kv, a.Skv - k0);
+    __syncthreads();
+    if (is_doc)
+      for (int c = threadIdx.x; c < cols; c += blockDim.x) doc_k[c] = a.doc_id[k0 + c];
+    __syncthreads();
+    bool any = false, all = true;
+    const int pairs = rows * cols;
+    for (int e = threadIdx.x; e < pairs; e += blockDim.x) {
+      const int r = e / cols, c = e % cols;
+      const bool ok = mask_allows(a, q0 + r, k0 + c, is_doc ? doc_q[r] : 0, doc_k, c);
+      any |= ok;
+      all &= ok;
+    }
+    const int any_b = __syncthreads_or(any);
+    const int all_b = __syncthreads_and(all);
+    if (threadIdx.x == 0) {
+      const uint8_t c = any_b ? (all_b ? 2 : 1) : 0;
+      a.cls[(int64_t)qt * a.nK + kt] = c;
+      if (c == 1) a.part_idx[(int64_t)qt * a.nK + np++] = kt;
+      if (c == 2) a.full_idx[(int64_t)qt * a.nK + nf++] = kt;
+    }
+  }
+  if (threadIdx.x == 0) {
+    a.part_cnt[qt] = np;
+    a.full_cnt[qt] = nf;
+  }
+}
+
+// One warp per output row: lse = ln sum_i exp(lse_i); o = sum_i exp(lse_i - lse) o_i.
+struct CombineArgs {
+  const float* o_parts;    // [rows][n][D]
+  const float* lse_parts;  // [rows][n]
+  int rows, n, D;
+  int rows_per_b;          // rows are (b, h) with h < rows_per_b
+  __nv_bfloat16* o;
+  int64_t o_sb, o_sh;      // element strides of the output rows (b, h)
+  float* lse;              // [rows] or nullptr
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) lse_combine_kernel(const CombineArgs a) {
+  const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= a.rows) return;
+  const float* lp = a.lse_parts + (int64_t)row * a.n;
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  float mx = NEG_INF;
+  for (int i = lane; i < a.n; i += 32) mx = fmaxf(mx, lp[i]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float sum = 0.f;
+  if (mx != NEG_INF)
+    for (int i = lane; i < a.n; i += 32) sum += expf(lp[i] - mx);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  const float lse = mx == NEG_INF ? NEG_INF : mx + logf(sum);
+  constexpr int V = D / 32;  // elements per lane
+  float acc[V];
+#pragma unroll
+  for (int j = 0; j < V; ++j) acc[j] = 0.f;
+  if (mx != NEG_INF) {
+    const float* op = a.o_parts + (int64_t)row * a.n * D + lane * V;
+    for (int i = 0; i < a.n; ++i) {
+      const float li = lp[i];
+      if (li == NEG_INF) continue;
+      const float wgt = expf(li - lse);
+      if constexpr (V == 4) {
+        const float4 f = *reinterpret_cast<const float4*>(op + (int64_t)i * D);
+        acc[0] += wgt * f.x;
+        acc[1] += wgt * f.y;
+        acc[2] += wgt * f.z;
+        acc[3] += wgt * f.w;
+      } else {
+        const float2 f = *reinterpret_cast<const float2*>(op + (int64_t)i * D);
+        acc[0] += wgt * f.x;
+        acc[1] += wgt * f.y;
+      }
+    }
+  }
+  const int b = row / a.rows_per_b, h = row % a.rows_per_b;
+  __nv_bfloat16* dst = a.o + (int64_t)b * a.o_sb + (int64_t)h * a.o_sh + lane * V;
+  if constexpr (V == 4) {
+    __nv_bfloat162 p0 = __floats2bfloat162_rn(acc[0], acc[1]);
+    __nv_bfloat162 p1 = __floats2bfloat162_rn(acc[2], acc[3]);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&p0);
+    u.y = *reinterpret_cast<uint32_t*>(&p1);
+    *reinterpret_cast<uint2*>(dst) = u;
+  } else {
+    *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(acc[0], acc[1]);
+  }
+  if (lane == 0 && a.lse != nullptr) a.lse[row] = lse;
+}
+
+}  // namespace attn_kernels

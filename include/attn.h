@@ -1,0 +1,186 @@
+/*
+ * attn.h - C ABI of the B200 (sm_100a) exact-attention forward library.
+ *
+ * The library computes exact scaled-dot-product attention forward,
+ *     O = softmax(score_mod(scale * Q K^T) + mask) V,
+ * tile by tile with an online (running max / running sum) softmax, so the
+ * Sq x Skv score matrix never reaches device memory ("A Deep Dive into Flash
+ * Attention": sections "Tiling the Computation", "2. Online Softmax",
+ * "3. Weighted Sum of Values"). The options are those of flash_attn_func /
+ * flash_attn_with_kvcache (FlashAttention overview, "Examples": softmax_scale,
+ * causal, window_size, alibi_slopes, cache_seqlens, block_table) and the
+ * FlexAttention hooks (attention-gym issue 101 repro: mask_mod q_idx >= kv_idx,
+ * create_block_mask with BLOCK_SIZE; "FlexAttention + FlashAttention-4" talk:
+ * score mods ALiBi / softcap, masks causal / sliding window, block sparsity).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    allocates nothing, frees nothing and never synchronises the stream.
+ *  - `stream` is a cudaStream_t passed as void*; every launch goes on it.
+ *  - Argument checks run on the host before any launch and return a status;
+ *    no C++ exception crosses this boundary.
+ *  - Kernel-detected problems (a wait that timed out, a page id outside the
+ *    cache) are OR-ed into the optional device int `*status` (ATTN_DEV_* bits)
+ *    and never trap. The caller reads it when it chooses.
+ *  - Inputs are bf16 (raw 16-bit storage), accumulation is fp32, O is bf16,
+ *    LSE is fp32 natural-log.
+ *  - Element strides are in elements; the head dimension is contiguous. Every
+ *    non-unit stride must be a multiple of 8 elements (16 bytes) and every
+ *    tensor base 16-byte aligned (a TMA requirement).
+ */
+#ifndef ATTN_H
+#define ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,  /* a pointer, size, stride or option is malformed */
+  ATTN_ERR_UNSUPPORTED = 2,  /* well-formed but outside what the kernels handle */
+  ATTN_ERR_CUDA = 3,         /* a CUDA runtime / driver call failed */
+  ATTN_ERR_WORKSPACE = 4     /* the caller's workspace is too small */
+} attn_status;
+
+/* Bits the kernels OR into *status. */
+#define ATTN_DEV_TIMEOUT 1   /* a bounded pipeline wait gave up; outputs invalid */
+#define ATTN_DEV_BAD_PAGE 2  /* a block_table entry was outside [0, num_pages) */
+
+/* Mask kinds (FlexAttention mask_mod equivalents, attention-gym issue 101 and
+ * the FA4 talk; flash_attn window_size in the FlashAttention overview).
+ * With q_pos = i + q_offset for query i and key position j:
+ *   NONE      every key allowed
+ *   CAUSAL    j <= q_pos                                   (q_idx >= kv_idx)
+ *   WINDOW    (left < 0 || q_pos - j <= left) && (right < 0 || j - q_pos <= right)
+ *   DOCUMENT  j <= q_pos && doc_id[i] == doc_id[j]   (packed sequences; Sq == Skv,
+ *             q_offset == 0; needs a block mask built from the same spec) */
+typedef enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_WINDOW = 2, ATTN_MASK_DOCUMENT = 3 } attn_mask_kind;
+
+/* Score modifiers applied to the scaled score s = scale * q.k before masking
+ * (FA4 talk, score_mod hooks; flash_attn alibi_slopes and softcapping):
+ *   SOFTCAP   s -> softcap * tanh(s / softcap)
+ *   ALIBI     s -> s + slope[b][h] * (j - q_pos)                                */
+typedef enum { ATTN_MOD_NONE = 0, ATTN_MOD_SOFTCAP = 1, ATTN_MOD_ALIBI = 2 } attn_mod_kind;
+
+typedef struct {
+  attn_mask_kind kind;
+  int window_left;        /* WINDOW: keys at most this far behind; -1 = unbounded */
+  int window_right;       /* WINDOW: keys at most this far ahead;  -1 = unbounded */
+  int q_offset;           /* position of query 0 on the key axis (CAUSAL / WINDOW) */
+  const int32_t *doc_id;  /* DOCUMENT: device int32 [S] document id per position */
+} attn_mask_spec;
+
+/* Block mask (FlexAttention create_block_mask equivalent): per (q-tile,
+ * kv-tile) class 0 = empty (skipped), 1 = partial (mask evaluated per
+ * element), 2 = full (no mask work), and per q-tile the ascending kv-tile
+ * lists of partial and full tiles. Broadcast over batch and heads. All arrays
+ * live inside one caller-owned device buffer laid out by attn_block_mask_layout. */
+typedef struct {
+  int Sq, Skv, blk_q, blk_kv, n_q_tiles, n_kv_tiles;
+  uint8_t *cls;       /* [n_q_tiles][n_kv_tiles] */
+  int32_t *part_cnt;  /* [n_q_tiles] */
+  int32_t *part_idx;  /* [n_q_tiles][n_kv_tiles], first part_cnt[q] entries valid */
+  int32_t *full_cnt;  /* [n_q_tiles] */
+  int32_t *full_idx;  /* [n_q_tiles][n_kv_tiles], first full_cnt[q] entries valid */
+} attn_block_mask;
+
+/* Bytes of device memory a block mask for these sizes needs (0 if invalid). */
+size_t attn_block_mask_bytes(int Sq, int Skv, int blk_q, int blk_kv);
+
+/* Carves the tables out of `buf` (device, >= attn_block_mask_bytes, 16-byte
+ * aligned) and fills `out`. Host-only pointer arithmetic; nothing is launched. */
+attn_status attn_block_mask_layout(void *buf, size_t buf_bytes, int Sq, int Skv, int blk_q, int blk_kv,
+                                   attn_block_mask *out);
+
+/* Classifies every tile of the mask on the device by evaluating the mask on
+ * each in-range (q, kv) pair (out-of-range positions of ragged edge tiles do
+ * not count) and writes the class table and both ascending index lists.
+ * Any mask kind is accepted; blk_q and blk_kv must be multiples of 16. */
+attn_status attn_build_block_mask(const attn_mask_spec *spec, const attn_block_mask *out, void *stream);
+
+typedef struct {
+  const void *q;              /* bf16 [B][Sq][Hq][D] via q_stride */
+  const void *k;              /* bf16 [B][Skv][Hkv][D] via k_stride */
+  const void *v;              /* bf16 [B][Skv][Hkv][D] via v_stride */
+  void *o;                    /* bf16 [B][Sq][Hq][D] via o_stride (output) */
+  float *lse;                 /* fp32 [B][Hq][Sq] contiguous (output); may be NULL */
+  int64_t q_stride[3];        /* element strides of batch, sequence, head */
+  int64_t k_stride[3];
+  int64_t v_stride[3];
+  int64_t o_stride[3];
+  int B, Hq, Hkv, Sq, Skv, D; /* Hq % Hkv == 0 (GQA/MQA without repeat_kv); D in {64, 128} */
+  float scale;                /* softmax_scale; <= 0 selects 1/sqrt(D) */
+  attn_mask_spec mask;
+  const attn_block_mask *block_mask; /* optional for NONE/CAUSAL/WINDOW, required for
+                                        DOCUMENT; 128 x 128 tiles built for (Sq, Skv) */
+  attn_mod_kind mod;
+  float softcap;              /* SOFTCAP: cap > 0 */
+  const float *alibi_slopes;  /* ALIBI: device fp32 [Hq] or [B][Hq] */
+  int alibi_batch_stride;     /* 0 for [Hq], Hq for [B][Hq] */
+  int *status;                /* optional device int, ATTN_DEV_* bits OR-ed in */
+} attn_fwd_params;
+
+/* Prefill / full-sequence forward: O and LSE for every query row. Empty
+ * tiles are skipped, full tiles do no mask work. Rows with no allowed key get
+ * O = 0 and LSE = -inf. Sq == 0 or B == 0 launches nothing. */
+attn_status attn_fwd(const attn_fwd_params *p, void *stream);
+
+typedef struct {
+  const void *q;              /* bf16 [B][Hq][D] (one new token per sequence) via q_stride */
+  int64_t q_stride[2];        /* element strides of batch, head */
+  const void *k_cache;        /* bf16 [num_pages][page_size][Hkv][D] via cache_stride */
+  const void *v_cache;        /* same shape and strides as k_cache */
+  int64_t cache_stride[3];    /* element strides of page, slot, head */
+  const int32_t *block_table; /* int32 [B][block_table_stride]: logical page -> physical page */
+  int block_table_stride;     /* >= max pages any sequence uses */
+  const int32_t *cache_seqlens; /* int32 [B]: keys of sequence b are its first cache_seqlens[b] tokens */
+  int B, Hq, Hkv, D, page_size, num_pages;
+  int max_seqlen;             /* upper bound on every cache_seqlens[b] (sizes the split) */
+  float scale;                /* <= 0 selects 1/sqrt(D) */
+  attn_mod_kind mod;          /* the query sits at position cache_seqlens[b] - 1 */
+  float softcap;
+  const float *alibi_slopes;
+  int alibi_batch_stride;
+  int num_splits;             /* key-axis splits per sequence; 0 = choose automatically */
+  void *o;                    /* bf16 [B][Hq][D] via o_stride (output) */
+  int64_t o_stride[2];
+  float *lse;                 /* fp32 [B][Hq] contiguous (output); may be NULL */
+  int *status;                /* optional device int, ATTN_DEV_* bits */
+} attn_decode_params;
+
+/* Number of splits attn_decode uses for these sizes (resolves num_splits = 0). */
+int attn_decode_num_splits(int B, int Hq, int Hkv, int max_seqlen, int num_splits);
+
+/* Workspace bytes attn_decode needs: one fp32 partial O row and LSE per
+ * (sequence, query head, split). */
+size_t attn_decode_workspace_bytes(int B, int Hq, int D, int num_splits);
+
+/* Split-KV decode over a paged KV cache (flash_attn_with_kvcache with
+ * block_table and cache_seqlens, FlashAttention overview, "Examples"): each
+ * (sequence, KV head, split) runs the online softmax over its share of the
+ * keys with all query heads of the group as the MMA rows and writes a partial
+ * (O_i, LSE_i); a second kernel combines them, LSE = ln sum_i exp(LSE_i) and
+ * O = sum_i exp(LSE_i - LSE) O_i. page_size must be a multiple of 16 that
+ * divides 128 or is a multiple of 128. `workspace` is caller-owned device
+ * memory of at least attn_decode_workspace_bytes(B, Hq, D, splits). */
+attn_status attn_decode(const attn_decode_params *p, void *workspace, size_t workspace_bytes, void *stream);
+
+/* The combine step on its own: merges n_splits partial results per row.
+ * o_parts fp32 [rows][n_splits][D] (normalised partial outputs), lse_parts fp32
+ * [rows][n_splits] (natural log, -inf = empty part); writes o bf16
+ * [rows][D] with row stride o_row_stride (elements) and lse fp32 [rows]
+ * (may be NULL). D in {64, 128}. */
+attn_status attn_lse_combine(const float *o_parts, const float *lse_parts, int rows, int n_splits, int D, void *o,
+                             int64_t o_row_stride, float *lse, void *stream);
+
+const char *attn_status_str(attn_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H */
