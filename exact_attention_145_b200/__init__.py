@@ -11,6 +11,8 @@ Entry points (same names as the C ABI):
   attn_decode(q, k_cache, ...)      split-KV paged decode          -> (O, LSE)
   attn_build_block_mask(...)        FlexAttention-style block mask -> BlockMask
   attn_lse_combine(o_parts, ...)    merge split partial results    -> (O, LSE)
+  attn_decode_noalloc(q, ...)       attn_decode for callers that cannot allocate
+                                    device memory (scratch inside the library)
 """
 from __future__ import annotations
 
@@ -21,7 +23,8 @@ from . import _lib
 from ._lib import (ATTN_DEV_BAD_PAGE, ATTN_DEV_TIMEOUT, MASK_CAUSAL, MASK_DOCUMENT, MASK_NONE, MASK_WINDOW,
                    MOD_ALIBI, MOD_NONE, MOD_SOFTCAP, AttnError)
 
-__all__ = ["attn_fwd", "attn_decode", "attn_build_block_mask", "attn_lse_combine", "BlockMask", "AttnError",
+__all__ = ["attn_fwd", "attn_decode", "attn_decode_noalloc", "attn_build_block_mask", "attn_lse_combine",
+           "BlockMask", "AttnError",
            "load_library", "ATTN_DEV_TIMEOUT", "ATTN_DEV_BAD_PAGE"]
 
 
@@ -243,6 +246,36 @@ def attn_decode(q, k_cache, v_cache, block_table, cache_seqlens, *, max_seqlen: 
     h = _stream_handle(q.device) if stream is None else stream
     _lib.check(lib.attn_decode(ctypes.byref(p), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                h), "attn_decode")
+    return out, lse
+
+
+def attn_decode_noalloc(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, *, max_seqlen: int,
+                        scale: Optional[float] = None, num_splits: int = 0, status=None, stream=None):
+    """attn_decode whose split partials live in a fixed 32 MiB array inside the
+    library, for callers that may not allocate device memory (out and lse are
+    the caller's). Calls that would need more scratch raise AttnError
+    (workspace too small). The first call on a device should precede any
+    stream capture; calls that overlap on the GPU share the array and race."""
+    if q.dim() == 4:
+        q = q[:, 0]
+    p = _lib.DecodeParams()
+    p.q = q.data_ptr()
+    p.q_stride = _lib.c_i64x2(q.stride(0), q.stride(1))
+    p.k_cache, p.v_cache = k_cache.data_ptr(), v_cache.data_ptr()
+    p.cache_stride = _lib.c_i64x3(*k_cache.stride()[:3])
+    p.block_table, p.block_table_stride = block_table.data_ptr(), block_table.stride(0)
+    p.cache_seqlens = cache_seqlens.data_ptr()
+    p.B, p.Hq, p.D = q.shape
+    p.num_pages, p.page_size, p.Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    p.max_seqlen = int(max_seqlen)
+    p.scale = 0.0 if scale is None else float(scale)
+    p.num_splits = int(num_splits)
+    p.o = out.data_ptr()
+    p.o_stride = _lib.c_i64x2(out.stride(0), out.stride(1))
+    p.lse = _ptr(lse)
+    p.status = _ptr(status)
+    h = _stream_handle(q.device) if stream is None else stream
+    _lib.check(_lib.load().attn_decode_noalloc(ctypes.byref(p), h), "attn_decode_noalloc")
     return out, lse
 
 

@@ -177,6 +177,26 @@ attn_status attn_decode(const attn_decode_params *p, void *workspace, size_t wor
 attn_status attn_lse_combine(const float *o_parts, const float *lse_parts, int rows, int n_splits, int D, void *o,
                              int64_t o_row_stride, float *lse, void *stream);
 
+/* attn_decode without a caller-provided workspace. The paper has no
+ * counterpart: this exists for callers that are not allowed to allocate
+ * device memory (a plugin that is handed only its inputs and outputs by an
+ * engine that plans all device memory up front, or a latency-critical loop
+ * that cannot risk cudaMalloc's device-wide synchronisation). The split
+ * partials live in a fixed array inside the library, ATTN_DECODE_NOALLOC_MAX_BYTES
+ * per device, held by every GPU that loads the library until exit.
+ *  - Same parameters and results as attn_decode.
+ *  - Returns ATTN_ERR_WORKSPACE, launching nothing, when the call's partials
+ *    (attn_decode_workspace_bytes for its B, Hq, D and split count) exceed the
+ *    maximum; pass a smaller num_splits or batch, or use attn_decode.
+ *  - The first call on a device looks up the array's device address (and may
+ *    load the device code); make it before any stream capture on that device.
+ *  - All calls on a device share the array and leave their partials in it;
+ *    nothing needs clearing, but calls that overlap on the GPU race, so keep
+ *    them ordered on one stream.
+ *  - Allocates and frees nothing. */
+#define ATTN_DECODE_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
+attn_status attn_decode_noalloc(const attn_decode_params *p, void *stream);
+
 const char *attn_status_str(attn_status s);
 
 #ifdef __cplusplus
