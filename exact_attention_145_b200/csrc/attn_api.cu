@@ -65,9 +65,9 @@ attn_status make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
 
 // The dynamic shared-memory opt-in is per device; remember which devices
 // have it for each kernel instantiation.
-template <int D, bool DECODE>
-attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdArgs& a,
-                       int grid, cudaStream_t stream) {
+template <int D, bool DECODE, int MOD>
+attn_status launch_fwd_mod(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdArgs& a,
+                           int grid, cudaStream_t stream) {
   using L = Layout<D, DECODE>;
   static std::mutex mu;
   static uint64_t ready_mask = 0;
@@ -76,14 +76,41 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!(ready_mask & (1ull << dev))) {
-      if (cudaFuncSetAttribute(attn_fwd_kernel<D, DECODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(attn_fwd_kernel<D, DECODE, MOD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                L::kSmemBytes) != cudaSuccess)
         return ATTN_ERR_CUDA;
       ready_mask |= 1ull << dev;
     }
   }
-  attn_fwd_kernel<D, DECODE><<<grid, kThreads, L::kSmemBytes, stream>>>(mq, mk, mv, a);
+  attn_fwd_kernel<D, DECODE, MOD><<<grid, kThreads, L::kSmemBytes, stream>>>(mq, mk, mv, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// One kernel per score mod keeps each instantiation's hot loop small.
+template <int D, bool DECODE>
+attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdArgs& a,
+                       int grid, cudaStream_t stream) {
+  switch (a.mod) {
+    case MOD_SOFTCAP:
+      return launch_fwd_mod<D, DECODE, MOD_SOFTCAP>(mq, mk, mv, a, grid, stream);
+    case MOD_ALIBI:
+      return launch_fwd_mod<D, DECODE, MOD_ALIBI>(mq, mk, mv, a, grid, stream);
+    default:
+      return launch_fwd_mod<D, DECODE, MOD_NONE>(mq, mk, mv, a, grid, stream);
+  }
+}
+
+// Streaming multiprocessors of the current device (persistent grid size).
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
 }
 
 bool strides_ok(const int64_t* s, int n) {
@@ -280,8 +307,10 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
   if (attn_status st = make_map(&mv, p->Skv > 0 ? p->v : p->q, 4, dk, sv2, kKeys, 1)) return st;
 
   const int HU = a.pair_heads ? a.Hq / 2 : a.Hq;
-  const long grid = (long)a.B * HU * a.n_row_units;
-  if (grid <= 0 || grid > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+  const long units = (long)a.B * HU * a.n_row_units;
+  if (units <= 0 || units > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+  a.n_units = (int)units;
+  const long grid = units < sm_count() ? units : sm_count();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return p->D == 128 ? launch_fwd<128, false>(mq, mk, mv, a, (int)grid, s)
                      : launch_fwd<64, false>(mq, mk, mv, a, (int)grid, s);
@@ -390,8 +419,10 @@ attn_status attn_decode(const attn_decode_params* p, void* workspace, size_t wor
   if (attn_status st = make_map(&mv, p->v_cache, 4, dc, sc, (uint32_t)a.box_rows, 2)) return st;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const long grid = (long)p->B * p->Hkv * splits;
-  if (grid > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+  const long units = (long)p->B * p->Hkv * splits;
+  if (units > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+  a.n_units = (int)units;
+  const long grid = units < sm_count() ? units : sm_count();
   attn_status st = p->D == 128 ? launch_fwd<128, true>(mq, mk, mv, a, (int)grid, s)
                                : launch_fwd<64, true>(mq, mk, mv, a, (int)grid, s);
   if (st != ATTN_OK) return st;
