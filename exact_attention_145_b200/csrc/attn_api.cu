@@ -209,8 +209,10 @@ attn_status attn_build_block_mask(const attn_mask_spec* spec, const attn_block_m
   a.part_idx = out->part_idx;
   a.full_cnt = out->full_cnt;
   a.full_idx = out->full_idx;
-  const size_t smem = (size_t)(a.blk_q + a.blk_kv) * sizeof(int);
-  build_block_mask_kernel<<<a.nQ, kMaskThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t smem = a.kind == ATTN_MASK_DOCUMENT ? (size_t)kKvPerCta * a.blk_kv * sizeof(int) : 0;
+  classify_tiles_kernel<<<dim3(a.nQ, (a.nK + kKvPerCta - 1) / kKvPerCta), kMaskThreads, smem, st>>>(a);
+  compact_lists_kernel<<<a.nQ, 32, 0, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -232,11 +234,13 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
   const int nK = (p->Skv + kKeys - 1) / kKeys;
   if (p->mask.kind == ATTN_MASK_DOCUMENT) {
     if (!p->mask.doc_id || p->Sq != p->Skv || p->mask.q_offset != 0 || !p->block_mask) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(p->mask.doc_id)) return ATTN_ERR_UNSUPPORTED;  // read as int4 by the kernel
   }
   if (p->block_mask) {
     const attn_block_mask* bm = p->block_mask;
     if (bm->blk_q != kRows || bm->blk_kv != kKeys || bm->Sq != p->Sq || bm->Skv != p->Skv || !bm->cls ||
-        bm->n_q_tiles != nQ || bm->n_kv_tiles != nK)
+        bm->n_q_tiles != nQ || bm->n_kv_tiles != nK || !bm->part_cnt || !bm->part_idx || !bm->full_cnt ||
+        !bm->full_idx)
       return ATTN_ERR_INVALID_ARG;
   }
 
@@ -272,6 +276,12 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
   }
   a.doc_id = p->mask.doc_id;
   a.bm_cls = p->block_mask ? p->block_mask->cls : nullptr;
+  if (p->block_mask) {
+    a.bm_part_cnt = p->block_mask->part_cnt;
+    a.bm_part_idx = p->block_mask->part_idx;
+    a.bm_full_cnt = p->block_mask->full_cnt;
+    a.bm_full_idx = p->block_mask->full_idx;
+  }
   a.nQ = nQ;
   a.nK = nK;
   a.mod = p->mod;

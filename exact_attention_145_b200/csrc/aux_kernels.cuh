@@ -16,9 +16,14 @@ struct MaskArgs {
   int32_t *part_cnt, *part_idx, *full_cnt, *full_idx;
 };
 
-__device__ __forceinline__ bool mask_allows(const MaskArgs& a, int i, int j, int doc_i, const int* doc_j_smem,
-                                            int jl) {
-  const long q_pos = (long)i + a.q_offset;
+// Block-mask build, pass 1: classify tiles. CTA (q-tile, group of kKvPerCta
+// kv-tiles); each thread evaluates its query rows against every in-range key
+// of a tile (stopping early once it has seen both an allowed and a masked
+// pair), then block votes give "any allowed" and "all allowed".
+constexpr int kMaskThreads = 128;
+constexpr int kKvPerCta = 8;
+
+__device__ __forceinline__ bool pair_allowed(const MaskArgs& a, long q_pos, int j, int doc_i, int doc_j) {
   switch (a.kind) {
     case 0:
       return true;
@@ -27,52 +32,63 @@ __device__ __forceinline__ bool mask_allows(const MaskArgs& a, int i, int j, int
     case 2:
       return (a.wl < 0 || q_pos - j <= a.wl) && (a.wr < 0 || (long)j - q_pos <= a.wr);
     default:
-      return (long)j <= q_pos && doc_j_smem[jl] == doc_i;
+      return (long)j <= q_pos && doc_j == doc_i;
   }
 }
 
-// One CTA per q-tile. For every kv-tile the block evaluates the mask on all
-// in-range (q, kv) pairs of the tile, reduces "any allowed" and "all allowed"
-// with block-wide votes, and thread 0 appends the tile to the partial or full
-// list, so both lists come out in ascending kv order.
-constexpr int kMaskThreads = 256;
-
-__global__ void __launch_bounds__(kMaskThreads) build_block_mask_kernel(const MaskArgs a) {
-  extern __shared__ int doc_smem[];  // [blk_q] query doc ids, then [blk_kv] key doc ids
-  int* doc_q = doc_smem;
-  int* doc_k = doc_smem + a.blk_q;
+__global__ void __launch_bounds__(kMaskThreads) classify_tiles_kernel(const MaskArgs a) {
+  extern __shared__ int doc_k[];  // [kKvPerCta * blk_kv] key doc ids (document masks)
   const int qt = blockIdx.x;
+  const int kt0 = blockIdx.y * kKvPerCta;
+  const int kt1 = min(kt0 + kKvPerCta, a.nK);
   const int q0 = qt * a.blk_q;
   const int rows = min(a.blk_q, a.Sq - q0);
   const bool is_doc = a.kind == 3;
-  if (is_doc)
-    for (int r = threadIdx.x; r < rows; r += blockDim.x) doc_q[r] = a.doc_id[q0 + r];
-  int np = 0, nf = 0;
-  for (int kt = 0; kt < a.nK; ++kt) {
+  if (is_doc) {
+    const int k_first = kt0 * a.blk_kv, k_end = min(kt1 * a.blk_kv, a.Skv);
+    for (int c = threadIdx.x; c < k_end - k_first; c += blockDim.x) doc_k[c] = a.doc_id[k_first + c];
+  }
+  __syncthreads();
+  for (int kt = kt0; kt < kt1; ++kt) {
     const int k0 = kt * a.blk_kv;
     const int cols = min(a.blk_kv, a.Skv - k0);
-    __syncthreads();
-    if (is_doc)
-      for (int c = threadIdx.x; c < cols; c += blockDim.x) doc_k[c] = a.doc_id[k0 + c];
-    __syncthreads();
+    const int* dk = doc_k + (kt - kt0) * a.blk_kv;
     bool any = false, all = true;
-    const int pairs = rows * cols;
-    for (int e = threadIdx.x; e < pairs; e += blockDim.x) {
-      const int r = e / cols, c = e % cols;
-      const bool ok = mask_allows(a, q0 + r, k0 + c, is_doc ? doc_q[r] : 0, doc_k, c);
-      any |= ok;
-      all &= ok;
+    for (int r = threadIdx.x; r < rows && (all || !any); r += blockDim.x) {
+      const long q_pos = (long)(q0 + r) + a.q_offset;
+      const int di = is_doc ? a.doc_id[q0 + r] : 0;
+      for (int c = 0; c < cols; ++c) {
+        const bool ok = pair_allowed(a, q_pos, k0 + c, di, is_doc ? dk[c] : 0);
+        any |= ok;
+        all &= ok;
+        if (any && !all) break;
+      }
     }
     const int any_b = __syncthreads_or(any);
     const int all_b = __syncthreads_and(all);
-    if (threadIdx.x == 0) {
-      const uint8_t c = any_b ? (all_b ? 2 : 1) : 0;
-      a.cls[(int64_t)qt * a.nK + kt] = c;
-      if (c == 1) a.part_idx[(int64_t)qt * a.nK + np++] = kt;
-      if (c == 2) a.full_idx[(int64_t)qt * a.nK + nf++] = kt;
-    }
+    if (threadIdx.x == 0) a.cls[(int64_t)qt * a.nK + kt] = any_b ? (all_b ? 2 : 1) : 0;
   }
-  if (threadIdx.x == 0) {
+}
+
+// Pass 2: one warp per q-tile compacts the class row into the ascending
+// partial and full lists with ballots.
+__global__ void __launch_bounds__(32) compact_lists_kernel(const MaskArgs a) {
+  const int qt = blockIdx.x;
+  const int lane = threadIdx.x;
+  const uint8_t* row = a.cls + (int64_t)qt * a.nK;
+  int np = 0, nf = 0;
+  for (int k0 = 0; k0 < a.nK; k0 += 32) {
+    const int kt = k0 + lane;
+    const uint8_t c = kt < a.nK ? row[kt] : 0;
+    const unsigned mp = __ballot_sync(0xffffffffu, c == 1);
+    const unsigned mf = __ballot_sync(0xffffffffu, c == 2);
+    const unsigned below = (1u << lane) - 1u;
+    if (c == 1) a.part_idx[(int64_t)qt * a.nK + np + __popc(mp & below)] = kt;
+    if (c == 2) a.full_idx[(int64_t)qt * a.nK + nf + __popc(mf & below)] = kt;
+    np += __popc(mp);
+    nf += __popc(mf);
+  }
+  if (lane == 0) {
     a.part_cnt[qt] = np;
     a.full_cnt[qt] = nf;
   }

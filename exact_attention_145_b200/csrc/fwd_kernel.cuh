@@ -71,6 +71,7 @@ struct FwdArgs {
   int mask, wl, wr, q_offset;
   const int32_t* doc_id;
   const uint8_t* bm_cls;  // [nQ][nK] class table or nullptr
+  const int32_t *bm_part_cnt, *bm_part_idx, *bm_full_cnt, *bm_full_idx;  // ascending kv-tile lists
   int nQ, nK;
   int mod;
   float softcap;
@@ -213,17 +214,30 @@ __device__ __forceinline__ int tile_class(const FwdArgs& a, const Work& w, int s
   }
 }
 
-// The key tiles a work unit visits. Prefill visits every kv tile that is
-// non-empty for either subtile, in ascending order: a contiguous range for the
-// analytic masks, a scan of the block-mask table otherwise. Decode step i
-// gives subtile s the tile t_begin + 2i + s.
-struct TileSeq {
-  int first;  // first tile (prefill) / t_begin (decode)
-  int n;      // number of steps
+// The key tiles a work unit visits, in ascending order. Prefill visits every
+// kv tile that is non-empty for either subtile: a contiguous range for the
+// analytic masks, the merge of the two subtiles' partial and full lists when
+// a block mask is given. Decode step i gives subtile s the tile t_begin+2i+s.
+struct TileWalker {
+  int t;  // current tile
+  // block-mask lists of the two subtiles' q-tiles (empty for an absent subtile)
+  const int32_t *p0, *f0, *p1, *f1;
+  int np0, nf0, np1, nf1, ip0, if0, ip1, if1;
 };
 
-__device__ __forceinline__ bool union_nonempty(const FwdArgs& a, const Work& w, int t) {
-  return (tile_class<false>(a, w, 0, t) | tile_class<false>(a, w, 1, t)) != 0;
+__device__ __forceinline__ int list_head(const int32_t* l, int n, int i) { return i < n ? __ldg(l + i) : 0x7fffffff; }
+
+__device__ __forceinline__ int walker_peek(const TileWalker& tw) {
+  return min(min(list_head(tw.p0, tw.np0, tw.ip0), list_head(tw.f0, tw.nf0, tw.if0)),
+             min(list_head(tw.p1, tw.np1, tw.ip1), list_head(tw.f1, tw.nf1, tw.if1)));
+}
+
+// Consumes tile t from every list whose head it is.
+__device__ __forceinline__ void walker_pop(TileWalker& tw, int t) {
+  if (list_head(tw.p0, tw.np0, tw.ip0) == t) ++tw.ip0;
+  if (list_head(tw.f0, tw.nf0, tw.if0) == t) ++tw.if0;
+  if (list_head(tw.p1, tw.np1, tw.ip1) == t) ++tw.ip1;
+  if (list_head(tw.f1, tw.nf1, tw.if1) == t) ++tw.if1;
 }
 
 // Tile range [lo, hi] of the window form q_pos - left <= kv <= q_pos + right
@@ -243,43 +257,62 @@ __device__ __forceinline__ bool subtile_range(const FwdArgs& a, const Work& w, i
   return true;
 }
 
+// Sets up the walk of one unit; returns the number of steps and leaves
+// tw.t on the first tile.
 template <bool DECODE>
-__device__ __forceinline__ TileSeq tile_seq(const FwdArgs& a, const Work& w) {
-  TileSeq ts;
+__device__ __forceinline__ int walker_init(const FwdArgs& a, const Work& w, TileWalker& tw) {
+  tw.np0 = tw.nf0 = tw.np1 = tw.nf1 = tw.ip0 = tw.if0 = tw.ip1 = tw.if1 = 0;
+  tw.p0 = tw.f0 = tw.p1 = tw.f1 = nullptr;
   if constexpr (DECODE) {
-    ts.first = w.t_begin;
-    ts.n = (w.t_end - w.t_begin + 1) / 2;
+    tw.t = w.t_begin;
+    return (w.t_end - w.t_begin + 1) / 2;
   } else if (a.bm_cls == nullptr) {
     int lo0 = 0, hi0 = -1, lo1 = 0, hi1 = -1;
     const bool e0 = subtile_range(a, w, 0, lo0, hi0), e1 = subtile_range(a, w, 1, lo1, hi1);
     if (!e0 && !e1) {
-      ts.first = 0;
-      ts.n = 0;
-    } else {
-      // the two subtile ranges overlap or touch (rows differ by at most one tile)
-      const int lo = e0 ? (e1 ? min(lo0, lo1) : lo0) : lo1;
-      const int hi = e0 ? (e1 ? max(hi0, hi1) : hi0) : hi1;
-      ts.first = lo;
-      ts.n = hi - lo + 1;
+      tw.t = 0;
+      return 0;
     }
+    // the two subtile ranges overlap or touch (rows differ by at most one tile)
+    const int lo = e0 ? (e1 ? min(lo0, lo1) : lo0) : lo1;
+    const int hi = e0 ? (e1 ? max(hi0, hi1) : hi0) : hi1;
+    tw.t = lo;
+    return hi - lo + 1;
   } else {
-    ts.first = a.nK;
-    ts.n = 0;
-    for (int t = a.nK - 1; t >= 0; --t)
-      if (union_nonempty(a, w, t)) {
-        ts.first = t;
-        ++ts.n;
-      }
+    if (w.row00 < a.Sq) {
+      const int qt = w.row00 / kRows;
+      tw.np0 = __ldg(a.bm_part_cnt + qt);
+      tw.nf0 = __ldg(a.bm_full_cnt + qt);
+      tw.p0 = a.bm_part_idx + (int64_t)qt * a.nK;
+      tw.f0 = a.bm_full_idx + (int64_t)qt * a.nK;
+    }
+    if (w.row01 < a.Sq && w.row01 != w.row00) {
+      const int qt = w.row01 / kRows;
+      tw.np1 = __ldg(a.bm_part_cnt + qt);
+      tw.nf1 = __ldg(a.bm_full_cnt + qt);
+      tw.p1 = a.bm_part_idx + (int64_t)qt * a.nK;
+      tw.f1 = a.bm_full_idx + (int64_t)qt * a.nK;
+    }
+    // count the union, then rewind
+    int n = 0;
+    TileWalker c = tw;
+    for (int t = walker_peek(c); t != 0x7fffffff; t = walker_peek(c)) {
+      walker_pop(c, t);
+      ++n;
+    }
+    tw.t = walker_peek(tw);
+    return n;
   }
-  return ts;
 }
 
-// Next prefill tile after t.
-__device__ __forceinline__ int next_tile(const FwdArgs& a, const Work& w, int t) {
-  ++t;
-  if (a.bm_cls != nullptr)
-    while (t < a.nK && !union_nonempty(a, w, t)) ++t;
-  return t;
+// Advances a prefill walk to the next tile.
+__device__ __forceinline__ void walker_next(const FwdArgs& a, TileWalker& tw) {
+  if (a.bm_cls == nullptr) {
+    ++tw.t;
+  } else {
+    walker_pop(tw, tw.t);
+    tw.t = walker_peek(tw);
+  }
 }
 
 // ---------------------------------------------------------------- producer
@@ -374,87 +407,122 @@ constexpr float kTanhA5 = 2.0f / 15.0f;
 constexpr float kTanhA7 = -17.0f / 315.0f;
 constexpr float kTanhA9 = 62.0f / 2835.0f;
 
-// Turns the raw scores of one row into log2-domain scores for the score mods.
-// softcap:  x = c*log2(e) * tanh(s*scale/c);  alibi: x = s*scale*log2(e) + slope*log2(e)*(kv - q_pos)
+// Score mods for one 32-column chunk of a row (chunk index c), turning raw
+// scores into log2-domain scores:
+//   softcap: x = c*log2(e) * tanh(s*scale/c);  alibi: x = s*scale*log2(e) + slope*log2(e)*(kv - q_pos)
 template <bool DECODE, int MOD>
-__device__ __forceinline__ void apply_score_mod(const FwdArgs& a, const Work& w, int s, int row, int t, float* x) {
+__device__ __forceinline__ void mod_chunk(const FwdArgs& a, const Work& w, int s, int row, int t, int c, float* x) {
   if constexpr (MOD == MOD_SOFTCAP) {
     const float k1 = a.scale / a.softcap;
     const float cl = a.softcap * kLog2e;
     float smax = 0.f;
 #pragma unroll
-    for (int c = 0; c < kKeys; c += 2) smax = max3(smax, fabsf(x[c]), fabsf(x[c + 1]));
+    for (int i = 0; i < 32; i += 2) smax = max3(smax, fabsf(x[i]), fabsf(x[i + 1]));
     if (smax * k1 <= kTanhPolyMax) {
       const float2 K1 = make_float2(k1, k1), CL = make_float2(cl, cl);
       const float2 A3 = make_float2(kTanhA3, kTanhA3), A5 = make_float2(kTanhA5, kTanhA5);
       const float2 A7 = make_float2(kTanhA7, kTanhA7), A9 = make_float2(kTanhA9, kTanhA9);
       const float2 ONE = make_float2(1.f, 1.f);
 #pragma unroll
-      for (int c = 0; c < kKeys; c += 2) {
-        const float2 y = mul2(make_float2(x[c], x[c + 1]), K1);
+      for (int i = 0; i < 32; i += 2) {
+        const float2 y = mul2(make_float2(x[i], x[i + 1]), K1);
         const float2 y2 = mul2(y, y);
         float2 q = fma2(y2, A9, A7);
         q = fma2(y2, q, A5);
         q = fma2(y2, q, A3);
         q = fma2(y2, q, ONE);
         const float2 r = mul2(mul2(y, CL), q);
-        x[c] = r.x;
-        x[c + 1] = r.y;
+        x[i] = r.x;
+        x[i + 1] = r.y;
       }
     } else {
-      // Some score of this row is large: tanh(y) = 1 - 2 / (e^{2y} + 1) on the SFU.
+      // Some score of this chunk is large: tanh(y) = 1 - 2 / (e^{2y} + 1) on the SFU.
       const float k2 = 2.0f * k1 * kLog2e;
 #pragma unroll
-      for (int c = 0; c < kKeys; ++c) x[c] = cl * (1.0f - 2.0f * rcp(ex2(x[c] * k2) + 1.0f));
+      for (int i = 0; i < 32; ++i) x[i] = cl * (1.0f - 2.0f * rcp(ex2(x[i] * k2) + 1.0f));
     }
   } else if constexpr (MOD == MOD_ALIBI) {
     const long q_pos = DECODE ? (long)w.seqlen - 1 : (long)(w_row0(w, s) + row) + a.q_offset;
     const int head = w_head(w, s) + (DECODE ? row : 0);
     const float slope = a.alibi[(int64_t)w.b * a.alibi_bstride + min(head, a.Hq - 1)] * kLog2e;
-    const float base = slope * (float)((long)t * kKeys - q_pos);
+    const float base = slope * (float)((long)t * kKeys + 32 * c - q_pos);
     const float2 SC = make_float2(a.scale_log2, a.scale_log2), SL = make_float2(slope, slope);
     const float2 B = make_float2(base, base);
 #pragma unroll
-    for (int c = 0; c < kKeys; c += 2) {
-      const float2 bias = fma2(SL, make_float2((float)c, (float)(c + 1)), B);
-      const float2 r = fma2(make_float2(x[c], x[c + 1]), SC, bias);
-      x[c] = r.x;
-      x[c + 1] = r.y;
+    for (int i = 0; i < 32; i += 2) {
+      const float2 bias = fma2(SL, make_float2((float)i, (float)(i + 1)), B);
+      const float2 r = fma2(make_float2(x[i], x[i + 1]), SC, bias);
+      x[i] = r.x;
+      x[i + 1] = r.y;
     }
   }
 }
 
-// Sets disallowed entries of a partial tile to -inf (works on raw or log2-domain scores).
+// Per-row mask bounds of one partial tile, computed once per step. Column
+// offset j (0..127) is allowed iff (unsigned)(j - clo) <= span, and for the
+// document mask also doc[kv0 + j] == dq.
+struct MaskRow {
+  int clo;
+  unsigned span;  // 0xffffffff sentinel handled by 'none'
+  bool none;
+  int dq;         // document id of the query row (document mask)
+};
+
 template <bool DECODE>
-__device__ __forceinline__ void apply_mask(const FwdArgs& a, const Work& w, int s, int row, int t, float* x) {
-  const float NEG_INF = -__int_as_float(0x7f800000);
+__device__ __forceinline__ MaskRow mask_row(const FwdArgs& a, const Work& w, int s, int row, int t) {
+  MaskRow m;
   const int kv0 = t * kKeys;
+  long lo, hi;
+  m.dq = 0;
   if constexpr (DECODE) {
-#pragma unroll
-    for (int c = 0; c < kKeys; ++c)
-      if (kv0 + c >= w.seqlen) x[c] = NEG_INF;
+    lo = 0;
+    hi = (long)w.seqlen - 1;
   } else {
     const int qrow = w_row0(w, s) + row;
     const long q_pos = (long)qrow + a.q_offset;
-    const int Skv = a.Skv;
     if (a.mask == MASK_DOCUMENT) {
-      const int dq = a.doc_id[min(qrow, a.Sq - 1)];
-#pragma unroll
-      for (int c = 0; c < kKeys; ++c) {
-        const int kv = kv0 + c;
-        const bool ok = kv < Skv && (long)kv <= q_pos && __ldg(a.doc_id + min(kv, Skv - 1)) == dq;
-        if (!ok) x[c] = NEG_INF;
-      }
+      lo = 0;
+      hi = q_pos;
+      m.dq = a.doc_id[min(qrow, a.Sq - 1)];
     } else {
-      // allowed iff lo <= kv <= hi, with kv < Skv; as offsets from kv0 in int
-      const long lo = a.wl >= 0 ? q_pos - a.wl : -(1l << 40);
-      const long hi = min(a.wr >= 0 ? q_pos + a.wr : (1l << 40), (long)Skv - 1);
-      const int clo = (int)max(min(lo - kv0, (long)kKeys), -1l);
-      const int chi = (int)max(min(hi - kv0, (long)kKeys), -1l);
-#pragma unroll
-      for (int c = 0; c < kKeys; ++c)
-        if (c < clo || c > chi) x[c] = NEG_INF;
+      lo = a.wl >= 0 ? q_pos - a.wl : -(1l << 40);
+      hi = a.wr >= 0 ? q_pos + a.wr : (1l << 40);
     }
+    hi = min(hi, (long)a.Skv - 1);
+  }
+  const long clo = max(lo - kv0, 0l), chi = min(hi - kv0, (long)kKeys - 1);
+  m.none = chi < clo;
+  m.clo = (int)min(clo, (long)kKeys);
+  m.span = m.none ? 0u : (unsigned)(chi - clo);
+  return m;
+}
+
+// Applies the mask to chunk c (columns 32c .. 32c+31) of a partial tile.
+template <bool DECODE>
+__device__ __forceinline__ void mask_chunk(const FwdArgs& a, const MaskRow& m, int t, int c, float* x) {
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  if (!DECODE && a.mask == MASK_DOCUMENT) {
+    const int kv = t * kKeys + 32 * c;
+    const int4* d4 = reinterpret_cast<const int4*>(a.doc_id + kv);
+    const int n4 = max(min(32, a.Skv - kv), 0) / 4;
+#pragma unroll
+    for (int i4 = 0; i4 < 8; ++i4) {
+      // volatile: keeps the load inside its chunk instead of letting all 32
+      // of a tile be hoisted (and spilled) ahead of the loop
+      int4 d = make_int4(-1, -1, -1, -1);
+      if (i4 < n4)
+        asm volatile("ld.global.nc.v4.s32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(d.x), "=r"(d.y), "=r"(d.z), "=r"(d.w)
+                     : "l"(d4 + i4));
+      const int j = 32 * c + 4 * i4;
+      x[4 * i4 + 0] = (!m.none && (unsigned)(j + 0 - m.clo) <= m.span && d.x == m.dq) ? x[4 * i4 + 0] : NEG_INF;
+      x[4 * i4 + 1] = (!m.none && (unsigned)(j + 1 - m.clo) <= m.span && d.y == m.dq) ? x[4 * i4 + 1] : NEG_INF;
+      x[4 * i4 + 2] = (!m.none && (unsigned)(j + 2 - m.clo) <= m.span && d.z == m.dq) ? x[4 * i4 + 2] : NEG_INF;
+      x[4 * i4 + 3] = (!m.none && (unsigned)(j + 3 - m.clo) <= m.span && d.w == m.dq) ? x[4 * i4 + 3] : NEG_INF;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = (!m.none && (unsigned)(32 * c + i - m.clo) <= m.span) ? x[i] : NEG_INF;
   }
 }
 
@@ -490,6 +558,64 @@ __device__ __forceinline__ float chunk_max(const float* x) {
   return max3(m0, m1, fmaxf(x[30], x[31]));
 }
 
+// Streams one tile out of TMEM 32 columns at a time: mods, mask (MASKED),
+// optimistic exponentials, P chunk stores. Returns the raw row max.
+template <bool DECODE, int MOD, bool MASKED>
+__device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, int s, int row, int t, uint32_t tS,
+                                             float* x, float nmu0, float2& acc0, float2& acc1) {
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  const float mult = MOD == MOD_NONE ? a.scale_log2 : 1.0f;
+  const float2 MULT = make_float2(mult, mult), NMU = make_float2(nmu0, nmu0);
+  MaskRow mr;
+  if constexpr (MASKED) mr = mask_row<DECODE>(a, w, s, row, t);
+  float mc = NEG_INF;
+  tmem_ld32f(tS, x);
+  tmem_ld_wait();
+  reg_fence_f<32>(x);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if (c < 3) tmem_ld32f(tS + 32 * (c + 1), x + 32 * (c + 1));
+    if constexpr (MOD != MOD_NONE) mod_chunk<DECODE, MOD>(a, w, s, row, t, c, x + 32 * c);
+    if constexpr (MASKED) mask_chunk<DECODE>(a, mr, t, c, x + 32 * c);
+    uint32_t pk[16];
+    exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
+    mc = fmaxf(mc, chunk_max(x + 32 * c));
+    tmem_st16(tS + 16 * c, pk);
+    if (c < 3) {
+      tmem_ld_wait();
+      reg_fence_f<32>(x + 32 * (c + 1));
+    }
+  }
+  return mc;
+}
+
+// First tile of a row: loads the scores chunk by chunk (the next chunk in
+// flight while this one gets its mods and mask) and returns the raw row max;
+// the exponentials follow once the max is known.
+template <bool DECODE, int MOD, bool MASKED>
+__device__ __forceinline__ float prepare_tile(const FwdArgs& a, const Work& w, int s, int row, int t, uint32_t tS,
+                                              float* x) {
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  MaskRow mr;
+  if constexpr (MASKED) mr = mask_row<DECODE>(a, w, s, row, t);
+  float mc = NEG_INF;
+  tmem_ld32f(tS, x);
+  tmem_ld_wait();
+  reg_fence_f<32>(x);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if (c < 3) tmem_ld32f(tS + 32 * (c + 1), x + 32 * (c + 1));
+    if constexpr (MOD != MOD_NONE) mod_chunk<DECODE, MOD>(a, w, s, row, t, c, x + 32 * c);
+    if constexpr (MASKED) mask_chunk<DECODE>(a, mr, t, c, x + 32 * c);
+    mc = fmaxf(mc, chunk_max(x + 32 * c));
+    if (c < 3) {
+      tmem_ld_wait();
+      reg_fence_f<32>(x + 32 * (c + 1));
+    }
+  }
+  return mc;
+}
+
 // One key tile of the online softmax for one query row (this thread's TMEM
 // lane). The exponentials are taken optimistically against the row's current
 // reference max while the scores stream in from TMEM chunk by chunk; only if
@@ -516,35 +642,22 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
     for (int j = 0; j < 32; ++j) pk[j] = 0u;
     tmem_st32(tS, pk);
     tmem_st32(tS + 32, pk);
-  } else if (MOD == MOD_NONE && cls == 2 && have_ref) {
-    // Streamed: chunk c+1 is in flight while chunk c is exponentiated.
-    const float2 NMU = make_float2(nmu0, nmu0);
-    float mc = NEG_INF;
-    tmem_ld32f(tS, x);
-    tmem_ld_wait();
-    reg_fence_f<32>(x);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (c < 3) tmem_ld32f(tS + 32 * (c + 1), x + 32 * (c + 1));
-      uint32_t pk[16];
-      exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
-      mc = fmaxf(mc, chunk_max(x + 32 * c));
-      tmem_st16(tS + 16 * c, pk);
-      if (c < 3) {
-        tmem_ld_wait();
-        reg_fence_f<32>(x + 32 * (c + 1));
-      }
-    }
-    mt = mc * mult;
+  } else if (MOD == MOD_NONE && have_ref) {
+    // Streamed: chunk c+1 is in flight while chunk c is (masked and)
+    // exponentiated against the current reference max. Full and partial
+    // tiles run separate instantiations so the common one stays compact.
+    if (cls == 2)
+      mt = stream_tile<DECODE, MOD, false>(a, w, s, row, t, tS, x, nmu0, acc0, acc1) * mult;
+    else
+      mt = stream_tile<DECODE, MOD, true>(a, w, s, row, t, tS, x, nmu0, acc0, acc1) * mult;
   } else {
-    tmem_ld128f(tS, x);
-    tmem_ld_wait();
-    reg_fence_f<kKeys>(x);
-    if constexpr (MOD != MOD_NONE) apply_score_mod<DECODE, MOD>(a, w, s, row, t, x);
-    if (cls == 1) apply_mask<DECODE>(a, w, s, row, t, x);
-    float mc = NEG_INF;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) mc = fmaxf(mc, chunk_max(x + 32 * c));
+    // Scores (with mods and mask) first; the exponentials follow against the
+    // reference max when there is one, else in the slow path below.
+    float mc;
+    if (cls == 2)
+      mc = prepare_tile<DECODE, MOD, false>(a, w, s, row, t, tS, x);
+    else
+      mc = prepare_tile<DECODE, MOD, true>(a, w, s, row, t, tS, x);
     mt = mc * mult;
     if (have_ref) {
       const float2 NMU = make_float2(nmu0, nmu0);
@@ -629,13 +742,11 @@ __device__ __forceinline__ bool epilogue(const FwdArgs& a, const Work& w, int s,
       }
       if (valid) {
 #pragma unroll
-        for (int j2 = 0; j2 < 32; j2 += 8) {
-          uint4 v4;
-          v4.x = pack_bf16x2(o[j2 + 0] * inv_l, o[j2 + 1] * inv_l);
-          v4.y = pack_bf16x2(o[j2 + 2] * inv_l, o[j2 + 3] * inv_l);
-          v4.z = pack_bf16x2(o[j2 + 4] * inv_l, o[j2 + 5] * inv_l);
-          v4.w = pack_bf16x2(o[j2 + 6] * inv_l, o[j2 + 7] * inv_l);
-          *reinterpret_cast<uint4*>(orow + c + j2) = v4;
+        for (int j2 = 0; j2 < 32; j2 += 16) {
+          uint32_t v8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v8[e] = pack_bf16x2(o[j2 + 2 * e] * inv_l, o[j2 + 2 * e + 1] * inv_l);
+          st_global_v8(orow + c + j2, v8);
         }
       }
     }
@@ -786,8 +897,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = unit_of(r);
       if (u < 0) continue;
       const Work w = map_work<DECODE>(a, u);
-      const TileSeq ts = tile_seq<DECODE>(a, w);
-      if (ts.n == 0) continue;
+      TileWalker tw;
+      const int n = walker_init<DECODE>(a, w, tw);
+      if (n == 0) continue;
       if (qcnt > 0 && !wait_all(&bar.q_empty, (qcnt - 1) & 1)) {
         ok = false;
         break;
@@ -805,9 +917,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       ++qcnt;
-      const int n_loads = DECODE ? 2 * ts.n : ts.n;
-      int t = ts.first;
+      const int n_loads = DECODE ? 2 * n : n;
       for (int k = 0; k < n_loads; ++k) {
+        const int t = tw.t;
         const int slot = kload % L::kNSlot;
         const int use = kload / L::kNSlot;
         if (use > 0 && !wait_all(&bar.kv_empty[slot], (use - 1) & 1)) {
@@ -821,7 +933,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   absent);
         __syncwarp();
         ++kload;
-        t = DECODE ? t + 1 : next_tile(a, w, t);
+        if (DECODE)
+          ++tw.t;
+        else
+          walker_next(a, tw);
       }
     }
     // Drain: on an abort, wait (bounded) for every copy still in flight so
@@ -847,7 +962,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t k_lo = sdesc_sw128_lo(smem_u32(smem + L::kKOff), 16);
     const uint32_t v_lo = sdesc_sw128_lo(smem_u32(smem + L::kVOff), L::kChunk);
     constexpr uint32_t kTileUnits = L::kTileBytes >> 4;
-    auto issue_qk = [&](int s, int slot) {
+    // last: the unit's final QK^T of subtile 1, after which Q may be reloaded.
+    auto issue_qk = [&](int s, int slot, bool last) {
       const uint32_t qa = q_lo + (DECODE ? 0u : (uint32_t)s * kTileUnits);
       const uint32_t ka = k_lo + (uint32_t)slot * kTileUnits;
       if (elect_one_sync()) {
@@ -857,6 +973,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + s * 128, sdesc_join(qa + off, kHi), sdesc_join(ka + off, kHi), idesc_qk, kk > 0);
         }
         mma_commit(&bar.s_ready[s]);
+        if (last) mma_commit(&bar.q_empty);
       }
       __syncwarp();
     };
@@ -869,17 +986,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = unit_of(r);
       if (u < 0) continue;
       const Work w = map_work<DECODE>(a, u);
-      const TileSeq ts = tile_seq<DECODE>(a, w);
-      const int n = ts.n;
+      TileWalker tw;
+      const int n = walker_init<DECODE>(a, w, tw);
       if (n == 0) continue;
       ok = wait_all(&bar.q_full, qcnt & 1);
       if (ok) ok = wait_all(&bar.k_full[slot_of(gstep, 0)], phase_of(gstep, 0));
       if (ok) {
         tc_fence_after();
-        issue_qk(0, slot_of(gstep, 0));
+        issue_qk(0, slot_of(gstep, 0), false);
         if (DECODE) ok = wait_all(&bar.k_full[slot_of(gstep, 1)], phase_of(gstep, 1));
         tc_fence_after();
-        if (ok) issue_qk(1, slot_of(gstep, 1));
+        if (ok) issue_qk(1, slot_of(gstep, 1), n == 1);
       }
       for (int j = 0; ok && j < n; ++j) {
         const int g = gstep + j;
@@ -900,14 +1017,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                      sdesc_join(va + ((kk * 16 * 128) >> 4), kHi), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
             if (!more) mma_commit(&bar.o_done[s]);
             if (DECODE || s == 1) mma_commit(&bar.kv_empty[slot]);
-            if (!more && s == 1) mma_commit(&bar.q_empty);  // every QK^T of the unit precedes
           }
           __syncwarp();
           if (more) {
             const int nslot = slot_of(g + 1, s);
             if (!wait_all(&bar.k_full[nslot], phase_of(g + 1, s))) { ok = false; break; }
             tc_fence_after();
-            issue_qk(s, nslot);
+            issue_qk(s, nslot, s == 1 && j + 2 == n);
           }
         }
       }
@@ -934,8 +1050,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = unit_of(r);
       if (u < 0) continue;
       const Work w = map_work<DECODE>(a, u);
-      const TileSeq ts = tile_seq<DECODE>(a, w);
-      const int n = ts.n;
+      TileWalker tw;
+      const int n = walker_init<DECODE>(a, w, tw);
       RowState st;
       st.m = -__int_as_float(0x7f800000);
       st.l = 0.f;
@@ -943,13 +1059,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         epilogue<D, DECODE>(a, w, s, row, lane_base, false, st, merge_m, merge_l, bar, qcnt, abort_flag);
         continue;
       }
-      int t = DECODE ? ts.first + s : ts.first;
+      if (DECODE) tw.t += s;
       for (int j = 0; j < n; ++j) {
+        const int t = tw.t;
         const int cls = tile_class<DECODE>(a, w, s, t);
         if (!wait_all(&bar.s_ready[s], (gstep + j) & 1)) { ok = false; break; }
         tc_fence_after();
         softmax_step<D, DECODE, MOD>(a, w, s, row, t, cls, tS, tO, j == 0, st, &bar.p_ready[s]);
-        t = DECODE ? t + 2 : next_tile(a, w, t);
+        if (DECODE)
+          tw.t += 2;
+        else
+          walker_next(a, tw);
       }
       if (!ok) break;
       bool got = wait_all(&bar.o_done[s], qcnt & 1);
