@@ -396,8 +396,11 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
                      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
-// Which of the 32 column pairs of a half-tile take the FMA-pipe exponential.
-__device__ __forceinline__ constexpr bool exp_on_fma(int j) { return (j % 16) >= 9; }
+// Which column pairs take the FMA-pipe exponential: 3 of every 16. The MUFU
+// pipe issues one ex2 per 8 cycles per warp; the polynomial costs a handful of
+// packed FMA-pipe ops per pair, so moving a small share off MUFU balances the two pipes
+// without starving the mask/max/convert work that also needs issue slots.
+__device__ __forceinline__ constexpr bool exp_on_fma(int j) { return (j % 16) >= 13; }
 
 // tanh on the FMA pipe for |y| <= kTanhPolyMax: the Taylor series
 // y - y^3/3 + 2y^5/15 - 17y^7/315 + 62y^9/2835 (tail below 1e-7 there).
@@ -560,12 +563,16 @@ __device__ __forceinline__ float chunk_max(const float* x) {
 
 // Streams one tile out of TMEM 32 columns at a time: mods, mask (MASKED),
 // optimistic exponentials, P chunk stores. Returns the raw row max.
+// With 'guess' set (the row has no reference max yet), the reference is taken
+// from chunk 0 of this tile and returned through ref_out (log2 units).
 template <bool DECODE, int MOD, bool MASKED>
 __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, int s, int row, int t, uint32_t tS,
-                                             float* x, float nmu0, float2& acc0, float2& acc1) {
+                                             float* x, float nmu0, float2& acc0, float2& acc1, bool guess,
+                                             float& ref_out) {
   const float NEG_INF = -__int_as_float(0x7f800000);
   const float mult = MOD == MOD_NONE ? a.scale_log2 : 1.0f;
-  const float2 MULT = make_float2(mult, mult), NMU = make_float2(nmu0, nmu0);
+  const float2 MULT = make_float2(mult, mult);
+  float2 NMU = make_float2(nmu0, nmu0);
   MaskRow mr;
   if constexpr (MASKED) mr = mask_row<DECODE>(a, w, s, row, t);
   float mc = NEG_INF;
@@ -577,9 +584,14 @@ __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, in
     if (c < 3) tmem_ld32f(tS + 32 * (c + 1), x + 32 * (c + 1));
     if constexpr (MOD != MOD_NONE) mod_chunk<DECODE, MOD>(a, w, s, row, t, c, x + 32 * c);
     if constexpr (MASKED) mask_chunk<DECODE>(a, mr, t, c, x + 32 * c);
+    mc = fmaxf(mc, chunk_max(x + 32 * c));
+    if (c == 0 && guess) {
+      const float g = mc * mult;
+      ref_out = g;
+      NMU = make_float2(g == NEG_INF ? 0.0f : -g, g == NEG_INF ? 0.0f : -g);
+    }
     uint32_t pk[16];
     exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
-    mc = fmaxf(mc, chunk_max(x + 32 * c));
     tmem_st16(tS + 16 * c, pk);
     if (c < 3) {
       tmem_ld_wait();
@@ -633,6 +645,7 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
   float mt;
   const bool have_ref = !first && __all_sync(0xffffffffu, st.m != NEG_INF);
   const float nmu0 = have_ref ? -st.m : 0.0f;
+  bool guessed = false;
   if (cls == 0) {
 #pragma unroll
     for (int c = 0; c < kKeys; ++c) x[c] = NEG_INF;
@@ -642,14 +655,27 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
     for (int j = 0; j < 32; ++j) pk[j] = 0u;
     tmem_st32(tS, pk);
     tmem_st32(tS + 32, pk);
-  } else if (MOD == MOD_NONE && have_ref) {
+  } else if (MOD == MOD_NONE) {
     // Streamed: chunk c+1 is in flight while chunk c is (masked and)
-    // exponentiated against the current reference max. Full and partial
-    // tiles run separate instantiations so the common one stays compact.
+    // exponentiated against the row's reference max; a row without one yet
+    // (first tile, or only masked keys so far) takes the max of its first
+    // chunk instead, corrected below if the tile exceeds it by more than the
+    // threshold. Full and partial tiles run separate instantiations so the
+    // common one stays compact.
+    const bool my_guess = first || st.m == NEG_INF;
+    float guess_ref = NEG_INF;
+    const float my_nmu = my_guess ? 0.0f : -st.m;
     if (cls == 2)
-      mt = stream_tile<DECODE, MOD, false>(a, w, s, row, t, tS, x, nmu0, acc0, acc1) * mult;
+      mt = stream_tile<DECODE, MOD, false>(a, w, s, row, t, tS, x, my_nmu, acc0, acc1, my_guess, guess_ref) * mult;
     else
-      mt = stream_tile<DECODE, MOD, true>(a, w, s, row, t, tS, x, nmu0, acc0, acc1) * mult;
+      mt = stream_tile<DECODE, MOD, true>(a, w, s, row, t, tS, x, my_nmu, acc0, acc1, my_guess, guess_ref) * mult;
+    if (my_guess) {
+      // This row's exponentials are relative to the guess, which becomes its
+      // reference; its l and O are still empty (or all zero).
+      st.m = guess_ref;
+      st.l = 0.0f;
+    }
+    guessed = true;
   } else {
     // Scores (with mods and mask) first; the exponentials follow against the
     // reference max when there is one, else in the slow path below.
@@ -669,8 +695,9 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
       }
     }
   }
-  // Slow path: first tile of the row, or a max that grew past the threshold.
-  const bool grow = !have_ref || mt > st.m + kRescaleThreshold;
+  // Slow path: no reference max yet (and none guessed), or a max that grew
+  // past the threshold.
+  const bool grow = (!have_ref && !guessed) || mt > st.m + kRescaleThreshold;
   float alpha = 1.0f;
   if (__any_sync(0xffffffffu, grow) && cls != 0) {
     const float m_new = fmaxf(st.m, mt);

@@ -71,7 +71,7 @@ typedef struct {
   int window_left;        /* WINDOW: keys at most this far behind; -1 = unbounded */
   int window_right;       /* WINDOW: keys at most this far ahead;  -1 = unbounded */
   int q_offset;           /* position of query 0 on the key axis (CAUSAL / WINDOW) */
-  const int32_t *doc_id;  /* DOCUMENT: device int32 [S] document id per position */
+  const int32_t *doc_id;  /* DOCUMENT: device int32 [S] document id per position, 16-byte aligned */
 } attn_mask_spec;
 
 /* Block mask (FlexAttention create_block_mask equivalent): per (q-tile,
