@@ -66,8 +66,8 @@ attn_status make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
 // The dynamic shared-memory opt-in is per device; remember which devices
 // have it for each kernel instantiation.
 template <int D, bool DECODE, int MOD>
-attn_status launch_fwd_mod(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdArgs& a,
-                           int grid, cudaStream_t stream) {
+attn_status launch_fwd_mod(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                           const FwdArgs& a, int grid, cudaStream_t stream) {
   using L = Layout<D, DECODE>;
   static std::mutex mu;
   static uint64_t ready_mask = 0;
@@ -82,21 +82,21 @@ attn_status launch_fwd_mod(const CUtensorMap& mq, const CUtensorMap& mk, const C
       ready_mask |= 1ull << dev;
     }
   }
-  attn_fwd_kernel<D, DECODE, MOD><<<grid, kThreads, L::kSmemBytes, stream>>>(mq, mk, mv, a);
+  attn_fwd_kernel<D, DECODE, MOD><<<grid, kThreads, L::kSmemBytes, stream>>>(mq, mk, mv, mo, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 // One kernel per score mod keeps each instantiation's hot loop small.
 template <int D, bool DECODE>
-attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdArgs& a,
-                       int grid, cudaStream_t stream) {
+attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                       const FwdArgs& a, int grid, cudaStream_t stream) {
   switch (a.mod) {
     case MOD_SOFTCAP:
-      return launch_fwd_mod<D, DECODE, MOD_SOFTCAP>(mq, mk, mv, a, grid, stream);
+      return launch_fwd_mod<D, DECODE, MOD_SOFTCAP>(mq, mk, mv, mo, a, grid, stream);
     case MOD_ALIBI:
-      return launch_fwd_mod<D, DECODE, MOD_ALIBI>(mq, mk, mv, a, grid, stream);
+      return launch_fwd_mod<D, DECODE, MOD_ALIBI>(mq, mk, mv, mo, a, grid, stream);
     default:
-      return launch_fwd_mod<D, DECODE, MOD_NONE>(mq, mk, mv, a, grid, stream);
+      return launch_fwd_mod<D, DECODE, MOD_NONE>(mq, mk, mv, mo, a, grid, stream);
   }
 }
 
@@ -116,6 +116,23 @@ int sm_count() {
 bool strides_ok(const int64_t* s, int n) {
   for (int i = 0; i < n; ++i)
     if (s[i] < 0 || (s[i] % 8) != 0) return false;
+  return true;
+}
+
+// Element strides [b, s, h] of a [B, S, H, D] tensor reordered to the tensor
+// map's (s, h, b) order. A size-1 dimension's stride is never used, so any
+// value there is replaced by one the encoder accepts; a zero stride on a
+// longer dimension (rows aliasing each other) is refused.
+bool map_strides(const int64_t* bsh, const uint64_t* dims, int64_t* out) {
+  const int64_t in[3] = {bsh[1], bsh[2], bsh[0]};
+  for (int i = 0; i < 3; ++i) {
+    if (dims[i + 1] == 1)
+      out[i] = in[i] > 0 ? in[i] : 8;
+    else if (in[i] > 0)
+      out[i] = in[i];
+    else
+      return false;
+  }
   return true;
 }
 
@@ -297,24 +314,20 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
   a.pair_heads = (a.g % 2 == 0) ? 1 : 0;
   a.n_row_units = a.pair_heads ? nQ : (nQ + 1) / 2;
 
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   const uint64_t dq[4] = {(uint64_t)p->D, (uint64_t)p->Sq, (uint64_t)p->Hq, (uint64_t)p->B};
-  const int64_t sq[3] = {p->q_stride[1], p->q_stride[2], p->q_stride[0]};
   // Skv == 0: every row is fully masked; the maps are never read (no tile is visited).
   const uint64_t dk[4] = {(uint64_t)p->D, (uint64_t)(p->Skv > 0 ? p->Skv : 1), (uint64_t)p->Hkv, (uint64_t)p->B};
-  const int64_t sk[3] = {p->k_stride[1], p->k_stride[2], p->k_stride[0]};
-  const int64_t sv[3] = {p->v_stride[1], p->v_stride[2], p->v_stride[0]};
-  // Degenerate strides of size-1 dims still have to pass the encoder's checks.
-  int64_t sq2[3], sk2[3], sv2[3];
-  for (int i = 0; i < 3; ++i) {
-    sq2[i] = sq[i] > 0 ? sq[i] : 8;
-    sk2[i] = sk[i] > 0 ? sk[i] : 8;
-    sv2[i] = sv[i] > 0 ? sv[i] : 8;
-  }
-  if (attn_status st = make_map(&mq, p->q, 4, dq, sq2, kRows, 1)) return st;
+  int64_t sq[3], sk[3], sv[3], so[3];
+  if (!map_strides(p->q_stride, dq, sq) || !map_strides(p->k_stride, dk, sk) || !map_strides(p->v_stride, dk, sv) ||
+      !map_strides(p->o_stride, dq, so))
+    return ATTN_ERR_UNSUPPORTED;
+  if (attn_status st = make_map(&mq, p->q, 4, dq, sq, kRows, 1)) return st;
   // With Skv == 0 nothing is read from K / V; the unused maps point at Q.
-  if (attn_status st = make_map(&mk, p->Skv > 0 ? p->k : p->q, 4, dk, sk2, kKeys, 1)) return st;
-  if (attn_status st = make_map(&mv, p->Skv > 0 ? p->v : p->q, 4, dk, sv2, kKeys, 1)) return st;
+  if (attn_status st = make_map(&mk, p->Skv > 0 ? p->k : p->q, 4, dk, sk, kKeys, 1)) return st;
+  if (attn_status st = make_map(&mv, p->Skv > 0 ? p->v : p->q, 4, dk, sv, kKeys, 1)) return st;
+  // O is written in 32-row boxes, one per softmax warp.
+  if (attn_status st = make_map(&mo, p->o, 4, dq, so, 32, 1)) return st;
 
   const int HU = a.pair_heads ? a.Hq / 2 : a.Hq;
   const long units = (long)a.B * HU * a.n_row_units;
@@ -322,8 +335,8 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
   a.n_units = (int)units;
   const long grid = units < sm_count() ? units : sm_count();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return p->D == 128 ? launch_fwd<128, false>(mq, mk, mv, a, (int)grid, s)
-                     : launch_fwd<64, false>(mq, mk, mv, a, (int)grid, s);
+  return p->D == 128 ? launch_fwd<128, false>(mq, mk, mv, mo, a, (int)grid, s)
+                     : launch_fwd<64, false>(mq, mk, mv, mo, a, (int)grid, s);
 }
 
 int attn_decode_num_splits(int B, int Hq, int Hkv, int max_seqlen, int num_splits) {
@@ -433,8 +446,9 @@ attn_status attn_decode(const attn_decode_params* p, void* workspace, size_t wor
   if (units > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
   a.n_units = (int)units;
   const long grid = units < sm_count() ? units : sm_count();
-  attn_status st = p->D == 128 ? launch_fwd<128, true>(mq, mk, mv, a, (int)grid, s)
-                               : launch_fwd<64, true>(mq, mk, mv, a, (int)grid, s);
+  // Decode writes fp32 partials with plain stores; its output map is unused.
+  attn_status st = p->D == 128 ? launch_fwd<128, true>(mq, mk, mv, mq, a, (int)grid, s)
+                               : launch_fwd<64, true>(mq, mk, mv, mq, a, (int)grid, s);
   if (st != ATTN_OK) return st;
   CombineArgs c;
   c.o_parts = a.part_o;

@@ -104,8 +104,16 @@ struct Layout {
   static constexpr int kKOff = kQOff + kNQ * kTileBytes;
   static constexpr int kVOff = kKOff + kNSlot * kTileBytes;
   static constexpr int kBarOff = kVOff + kNSlot * kTileBytes;
-  static constexpr int kSmemBytes = kBarOff + 1024 + 2 * 128 * 4 + 1024;  // + barriers + merge scratch + align slack
+  // After the barriers: decode's merge scratch (two 128-float rows), or
+  // prefill's output staging, one 32-row x 64-column bf16 SW128 box per
+  // softmax warp (the source of that warp's TMA stores).
+  static constexpr int kExtraOff = kBarOff + 1024;
+  static constexpr int kStageWarpBytes = 32 * 128;
+  static constexpr int kExtraBytes = DECODE ? 2 * 128 * 4 : 8 * kStageWarpBytes;
+  static constexpr int kSmemBytes = kExtraOff + kExtraBytes + 1024;  // + alignment slack
   static constexpr int kOCols = D;  // TMEM columns of one O accumulator
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+  static_assert(kExtraOff % 1024 == 0, "SW128 staging needs 1024-byte alignment");
 };
 
 struct Barriers {
@@ -500,7 +508,11 @@ __device__ __forceinline__ MaskRow mask_row(const FwdArgs& a, const Work& w, int
   return m;
 }
 
-// Applies the mask to chunk c (columns 32c .. 32c+31) of a partial tile.
+// Applies the mask to chunk c (columns 32c .. 32c+31) of a partial tile. For
+// the prefill window forms (causal included) the row's allowed range becomes
+// a 32-bit mask for the chunk, so each element costs one bit test and one
+// select; decode (only a split's ragged last tile) and the document mask keep
+// the range compare, which needs fewer live registers.
 template <bool DECODE>
 __device__ __forceinline__ void mask_chunk(const FwdArgs& a, const MaskRow& m, int t, int c, float* x) {
   const float NEG_INF = -__int_as_float(0x7f800000);
@@ -523,9 +535,15 @@ __device__ __forceinline__ void mask_chunk(const FwdArgs& a, const MaskRow& m, i
       x[4 * i4 + 2] = (!m.none && (unsigned)(j + 2 - m.clo) <= m.span && d.z == m.dq) ? x[4 * i4 + 2] : NEG_INF;
       x[4 * i4 + 3] = (!m.none && (unsigned)(j + 3 - m.clo) <= m.span && d.w == m.dq) ? x[4 * i4 + 3] : NEG_INF;
     }
-  } else {
+  } else if constexpr (DECODE) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) x[i] = (!m.none && (unsigned)(32 * c + i - m.clo) <= m.span) ? x[i] : NEG_INF;
+  } else {
+    const int lo = m.clo - 32 * c, hi = m.clo + (int)m.span - 32 * c;
+    unsigned bits = 0u;
+    if (!m.none && hi >= 0 && lo <= 31) bits = (0xffffffffu >> (31 - min(hi, 31))) & (0xffffffffu << max(lo, 0));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = (bits & (1u << i)) ? x[i] : NEG_INF;
   }
 }
 
@@ -744,37 +762,50 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
 // Epilogue of one unit for softmax subtile s: O / l to bf16 (prefill) or the
 // merged, normalised split partial (decode), and the LSE.
 template <int D, bool DECODE>
-__device__ __forceinline__ bool epilogue(const FwdArgs& a, const Work& w, int s, int row, uint32_t lane_base,
-                                         bool have_o, const RowState& st, float* merge_m, float* merge_l,
+__device__ __forceinline__ bool epilogue(const FwdArgs& a, const CUtensorMap* map_o, const Work& w, int s, int row,
+                                         uint32_t lane_base, bool have_o, const RowState& st, uint8_t* extra,
                                          Barriers& bar, int mcnt, volatile int* abort_flag) {
   using L = Layout<D, DECODE>;
   const float NEG_INF = -__int_as_float(0x7f800000);
   const uint32_t tO = lane_base + 256 + s * L::kOCols;
   if constexpr (!DECODE) {
-    const int qrow = w_row0(w, s) + row;
+    // Each warp writes its 32 rows as 64-column boxes: registers -> its SW128
+    // staging box in shared memory -> one TMA store per box, so the global
+    // writes are whole 128-byte lines instead of one row per lane.
+    const int wq = row / 32, lane = row % 32;
+    const int r0 = w_row0(w, s);
     const int h = w_head(w, s);
-    const bool valid = qrow < a.Sq && w_row0(w, s) < a.Sq;
+    const int qrow = r0 + row;
+    const bool valid = qrow < a.Sq && r0 < a.Sq;
+    const bool box_valid = r0 + 32 * wq < a.Sq;  // warp-uniform; rows past Sq are clipped by the map
     const float inv_l = st.l > 0.f ? 1.0f / st.l : 0.f;
-    __nv_bfloat16* orow = a.o + (int64_t)w.b * a.o_sb + (int64_t)qrow * a.o_ss + (int64_t)h * a.o_sh;
+    uint8_t* stage = extra + (s * 4 + wq) * L::kStageWarpBytes;
+    const uint32_t srow = smem_u32(stage) + lane * 128;
 #pragma unroll
-    for (int c = 0; c < D; c += 32) {
-      float o[32];
+    for (int hh = 0; hh < D / 64; ++hh) {
+      float o[64];
       if (have_o) {
-        tmem_ld32f(tO + c, o);
+        tmem_ld64f(tO + 64 * hh, o);
         tmem_ld_wait();
-        reg_fence_f<32>(o);
+        reg_fence_f<64>(o);
       } else {
 #pragma unroll
-        for (int j2 = 0; j2 < 32; ++j2) o[j2] = 0.f;
+        for (int j2 = 0; j2 < 64; ++j2) o[j2] = 0.f;
       }
-      if (valid) {
+      uint32_t pk[32];
 #pragma unroll
-        for (int j2 = 0; j2 < 32; j2 += 16) {
-          uint32_t v8[8];
+      for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
+      // The staging box is free once this warp's previous store has read it.
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v8[e] = pack_bf16x2(o[j2 + 2 * e] * inv_l, o[j2 + 2 * e + 1] * inv_l);
-          st_global_v8(orow + c + j2, v8);
-        }
+      for (int j = 0; j < 8; ++j)
+        st_shared_v4(srow + ((uint32_t)(j ^ (lane & 7)) << 4), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && box_valid) {
+        tma_store_4d(map_o, stage, 64 * hh, r0 + 32 * wq, h, w.b);
+        bulk_commit_group();
       }
     }
     if (valid && a.lse != nullptr)
@@ -787,6 +818,8 @@ __device__ __forceinline__ bool epilogue(const FwdArgs& a, const Work& w, int s,
     // normalised partial O_i and LSE_i of this split. The row stats of
     // subtile 1 are handed over through shared memory with two bounded
     // mbarrier handshakes (no named barrier, so an abort cannot hang here).
+    float* merge_m = reinterpret_cast<float*>(extra);
+    float* merge_l = merge_m + 128;
     float m1 = NEG_INF, l1v = 0.f;
     if (have_o) {
       if (s == 1) {
@@ -856,13 +889,13 @@ __device__ __forceinline__ bool epilogue(const FwdArgs& a, const Work& w, int s,
 template <int D, bool DECODE, int MOD>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                    const __grid_constant__ CUtensorMap map_v, const FwdArgs a) {
+                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
+                    const FwdArgs a) {
   using L = Layout<D, DECODE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Barriers& bar = *reinterpret_cast<Barriers*>(smem + L::kBarOff);
-  float* merge_m = reinterpret_cast<float*>(smem + L::kBarOff + 1024);
-  float* merge_l = merge_m + 128;
+  uint8_t* extra = smem + L::kExtraOff;
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   volatile int* abort_flag = &bar.abort_flag;
@@ -1083,7 +1116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       st.m = -__int_as_float(0x7f800000);
       st.l = 0.f;
       if (n == 0) {
-        epilogue<D, DECODE>(a, w, s, row, lane_base, false, st, merge_m, merge_l, bar, qcnt, abort_flag);
+        epilogue<D, DECODE>(a, &map_o, w, s, row, lane_base, false, st, extra, bar, qcnt, abort_flag);
         continue;
       }
       if (DECODE) tw.t += s;
@@ -1103,7 +1136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (DECODE && s == 0) got = got && wait_all(&bar.o_done[1], qcnt & 1);
       if (!got) break;
       tc_fence_after();
-      if (!epilogue<D, DECODE>(a, w, s, row, lane_base, true, st, merge_m, merge_l, bar, qcnt, abort_flag)) break;
+      if (!epilogue<D, DECODE>(a, &map_o, w, s, row, lane_base, true, st, extra, bar, qcnt, abort_flag)) break;
       // O is read: the next unit's first PV may overwrite it. In decode the
       // subtile-0 threads read both accumulators and release both.
       tc_fence_before();
@@ -1117,6 +1150,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++qcnt;
     }
     (void)tO;
+    // Output stores complete before the CTA (and its staging memory) goes away.
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
