@@ -65,7 +65,7 @@ attn_status make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
 
 // The dynamic shared-memory opt-in is per device; remember which devices
 // have it for each kernel instantiation.
-template <int D, bool DECODE, int MOD>
+template <int D, bool DECODE, int MOD, bool BM>
 attn_status launch_fwd_mod(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                            const FwdArgs& a, int grid, cudaStream_t stream) {
   using L = Layout<D, DECODE>;
@@ -76,28 +76,37 @@ attn_status launch_fwd_mod(const CUtensorMap& mq, const CUtensorMap& mk, const C
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!(ready_mask & (1ull << dev))) {
-      if (cudaFuncSetAttribute(attn_fwd_kernel<D, DECODE, MOD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(attn_fwd_kernel<D, DECODE, MOD, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                L::kSmemBytes) != cudaSuccess)
         return ATTN_ERR_CUDA;
       ready_mask |= 1ull << dev;
     }
   }
-  attn_fwd_kernel<D, DECODE, MOD><<<grid, kThreads, L::kSmemBytes, stream>>>(mq, mk, mv, mo, a);
+  attn_fwd_kernel<D, DECODE, MOD, BM><<<grid, kThreads, L::kSmemBytes, stream>>>(mq, mk, mv, mo, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// One kernel per score mod keeps each instantiation's hot loop small.
+// One kernel per score mod, and (prefill) per "block mask given or not",
+// keeps each instantiation's code small: code that runs once per work unit
+// (setup, masked tiles, epilogue) is otherwise evicted from the instruction
+// cache by the hot loop and refetched every unit.
+template <int D, bool DECODE, bool BM>
+attn_status launch_fwd_bm(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                          const FwdArgs& a, int grid, cudaStream_t stream) {
+  switch (a.mod) {
+    case MOD_SOFTCAP:
+      return launch_fwd_mod<D, DECODE, MOD_SOFTCAP, BM>(mq, mk, mv, mo, a, grid, stream);
+    case MOD_ALIBI:
+      return launch_fwd_mod<D, DECODE, MOD_ALIBI, BM>(mq, mk, mv, mo, a, grid, stream);
+    default:
+      return launch_fwd_mod<D, DECODE, MOD_NONE, BM>(mq, mk, mv, mo, a, grid, stream);
+  }
+}
 template <int D, bool DECODE>
 attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                        const FwdArgs& a, int grid, cudaStream_t stream) {
-  switch (a.mod) {
-    case MOD_SOFTCAP:
-      return launch_fwd_mod<D, DECODE, MOD_SOFTCAP>(mq, mk, mv, mo, a, grid, stream);
-    case MOD_ALIBI:
-      return launch_fwd_mod<D, DECODE, MOD_ALIBI>(mq, mk, mv, mo, a, grid, stream);
-    default:
-      return launch_fwd_mod<D, DECODE, MOD_NONE>(mq, mk, mv, mo, a, grid, stream);
-  }
+  if (!DECODE && a.bm_cls != nullptr) return launch_fwd_bm<D, DECODE, !DECODE>(mq, mk, mv, mo, a, grid, stream);
+  return launch_fwd_bm<D, DECODE, false>(mq, mk, mv, mo, a, grid, stream);
 }
 
 // Streaming multiprocessors of the current device (persistent grid size).

@@ -10,7 +10,9 @@
 //   warps 10-11 idle (they complete the third warpgroup for the register split)
 // The softmax warpgroups raise their register budget to kSoftmaxRegs and the
 // third warpgroup lowers its own to kControlRegs: 2*128*224 + 128*56 equals
-// the 384*168 registers the block is launched with.
+// the 384*168 registers the block is launched with. setmaxnreg acts on a whole
+// warpgroup: its four warps must all request the same count, so the idle
+// warps cannot give their share to the MMA and TMA warps.
 // The tensor pipe alternates between the subtiles so that one subtile's
 // softmax overlaps the other's MMAs: on B200 the exponentials take about
 // twice as long as the two GEMMs of a tile, so a single query tile per CTA
@@ -52,7 +54,7 @@ constexpr int kRows = 128;      // query rows per subtile (MMA M)
 constexpr int kKeys = 128;      // keys per K/V tile (MMA N of QK^T, K of PV)
 constexpr int kThreads = 384;
 constexpr int kSoftmaxRegs = 224;
-constexpr int kControlRegs = 56;
+constexpr int kControlRegs = 56;  // warps 8-11, one warpgroup, one count
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split exceeds launch budget");
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
@@ -184,8 +186,9 @@ __device__ __forceinline__ Work map_work(const FwdArgs& a, int u) {
   return w;
 }
 
-// Tile class of kv tile t for subtile s: 0 empty, 1 partial, 2 full.
-template <bool DECODE>
+// Tile class of kv tile t for subtile s: 0 empty, 1 partial, 2 full. BM:
+// the classes come from a block mask's table instead of the window bounds.
+template <bool DECODE, bool BM>
 __device__ __forceinline__ int tile_class(const FwdArgs& a, const Work& w, int s, int t) {
   if constexpr (DECODE) {
     (void)s;
@@ -199,7 +202,7 @@ __device__ __forceinline__ int tile_class(const FwdArgs& a, const Work& w, int s
     const int c1 = min(c0 + kKeys, a.Skv) - 1;
     const bool ragged = c0 + kKeys > a.Skv;
     int cls;
-    if (a.bm_cls != nullptr) {
+    if constexpr (BM) {
       cls = a.bm_cls[(r0 / kRows) * a.nK + t];
     } else if (a.mask == MASK_NONE) {
       cls = 2;
@@ -267,14 +270,14 @@ __device__ __forceinline__ bool subtile_range(const FwdArgs& a, const Work& w, i
 
 // Sets up the walk of one unit; returns the number of steps and leaves
 // tw.t on the first tile.
-template <bool DECODE>
+template <bool DECODE, bool BM>
 __device__ __forceinline__ int walker_init(const FwdArgs& a, const Work& w, TileWalker& tw) {
   tw.np0 = tw.nf0 = tw.np1 = tw.nf1 = tw.ip0 = tw.if0 = tw.ip1 = tw.if1 = 0;
   tw.p0 = tw.f0 = tw.p1 = tw.f1 = nullptr;
   if constexpr (DECODE) {
     tw.t = w.t_begin;
     return (w.t_end - w.t_begin + 1) / 2;
-  } else if (a.bm_cls == nullptr) {
+  } else if constexpr (!BM) {
     int lo0 = 0, hi0 = -1, lo1 = 0, hi1 = -1;
     const bool e0 = subtile_range(a, w, 0, lo0, hi0), e1 = subtile_range(a, w, 1, lo1, hi1);
     if (!e0 && !e1) {
@@ -314,8 +317,9 @@ __device__ __forceinline__ int walker_init(const FwdArgs& a, const Work& w, Tile
 }
 
 // Advances a prefill walk to the next tile.
-__device__ __forceinline__ void walker_next(const FwdArgs& a, TileWalker& tw) {
-  if (a.bm_cls == nullptr) {
+template <bool BM>
+__device__ __forceinline__ void walker_next(TileWalker& tw) {
+  if constexpr (!BM) {
     ++tw.t;
   } else {
     walker_pop(tw, tw.t);
@@ -479,7 +483,7 @@ struct MaskRow {
   int dq;         // document id of the query row (document mask)
 };
 
-template <bool DECODE>
+template <bool DECODE, bool BM>
 __device__ __forceinline__ MaskRow mask_row(const FwdArgs& a, const Work& w, int s, int row, int t) {
   MaskRow m;
   const int kv0 = t * kKeys;
@@ -491,7 +495,7 @@ __device__ __forceinline__ MaskRow mask_row(const FwdArgs& a, const Work& w, int
   } else {
     const int qrow = w_row0(w, s) + row;
     const long q_pos = (long)qrow + a.q_offset;
-    if (a.mask == MASK_DOCUMENT) {
+    if (BM && a.mask == MASK_DOCUMENT) {
       lo = 0;
       hi = q_pos;
       m.dq = a.doc_id[min(qrow, a.Sq - 1)];
@@ -513,10 +517,10 @@ __device__ __forceinline__ MaskRow mask_row(const FwdArgs& a, const Work& w, int
 // a 32-bit mask for the chunk, so each element costs one bit test and one
 // select; decode (only a split's ragged last tile) and the document mask keep
 // the range compare, which needs fewer live registers.
-template <bool DECODE>
+template <bool DECODE, bool BM>
 __device__ __forceinline__ void mask_chunk(const FwdArgs& a, const MaskRow& m, int t, int c, float* x) {
   const float NEG_INF = -__int_as_float(0x7f800000);
-  if (!DECODE && a.mask == MASK_DOCUMENT) {
+  if (BM && a.mask == MASK_DOCUMENT) {
     const int kv = t * kKeys + 32 * c;
     const int4* d4 = reinterpret_cast<const int4*>(a.doc_id + kv);
     const int n4 = max(min(32, a.Skv - kv), 0) / 4;
@@ -583,7 +587,7 @@ __device__ __forceinline__ float chunk_max(const float* x) {
 // optimistic exponentials, P chunk stores. Returns the raw row max.
 // With 'guess' set (the row has no reference max yet), the reference is taken
 // from chunk 0 of this tile and returned through ref_out (log2 units).
-template <bool DECODE, int MOD, bool MASKED>
+template <bool DECODE, int MOD, bool MASKED, bool BM>
 __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, int s, int row, int t, uint32_t tS,
                                              float* x, float nmu0, float2& acc0, float2& acc1, bool guess,
                                              float& ref_out) {
@@ -592,7 +596,7 @@ __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, in
   const float2 MULT = make_float2(mult, mult);
   float2 NMU = make_float2(nmu0, nmu0);
   MaskRow mr;
-  if constexpr (MASKED) mr = mask_row<DECODE>(a, w, s, row, t);
+  if constexpr (MASKED) mr = mask_row<DECODE, BM>(a, w, s, row, t);
   float mc = NEG_INF;
   tmem_ld32f(tS, x);
   tmem_ld_wait();
@@ -601,7 +605,7 @@ __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, in
   for (int c = 0; c < 4; ++c) {
     if (c < 3) tmem_ld32f(tS + 32 * (c + 1), x + 32 * (c + 1));
     if constexpr (MOD != MOD_NONE) mod_chunk<DECODE, MOD>(a, w, s, row, t, c, x + 32 * c);
-    if constexpr (MASKED) mask_chunk<DECODE>(a, mr, t, c, x + 32 * c);
+    if constexpr (MASKED) mask_chunk<DECODE, BM>(a, mr, t, c, x + 32 * c);
     mc = fmaxf(mc, chunk_max(x + 32 * c));
     if (c == 0 && guess) {
       const float g = mc * mult;
@@ -622,12 +626,12 @@ __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, in
 // First tile of a row: loads the scores chunk by chunk (the next chunk in
 // flight while this one gets its mods and mask) and returns the raw row max;
 // the exponentials follow once the max is known.
-template <bool DECODE, int MOD, bool MASKED>
+template <bool DECODE, int MOD, bool MASKED, bool BM>
 __device__ __forceinline__ float prepare_tile(const FwdArgs& a, const Work& w, int s, int row, int t, uint32_t tS,
                                               float* x) {
   const float NEG_INF = -__int_as_float(0x7f800000);
   MaskRow mr;
-  if constexpr (MASKED) mr = mask_row<DECODE>(a, w, s, row, t);
+  if constexpr (MASKED) mr = mask_row<DECODE, BM>(a, w, s, row, t);
   float mc = NEG_INF;
   tmem_ld32f(tS, x);
   tmem_ld_wait();
@@ -636,7 +640,7 @@ __device__ __forceinline__ float prepare_tile(const FwdArgs& a, const Work& w, i
   for (int c = 0; c < 4; ++c) {
     if (c < 3) tmem_ld32f(tS + 32 * (c + 1), x + 32 * (c + 1));
     if constexpr (MOD != MOD_NONE) mod_chunk<DECODE, MOD>(a, w, s, row, t, c, x + 32 * c);
-    if constexpr (MASKED) mask_chunk<DECODE>(a, mr, t, c, x + 32 * c);
+    if constexpr (MASKED) mask_chunk<DECODE, BM>(a, mr, t, c, x + 32 * c);
     mc = fmaxf(mc, chunk_max(x + 32 * c));
     if (c < 3) {
       tmem_ld_wait();
@@ -651,7 +655,7 @@ __device__ __forceinline__ float prepare_tile(const FwdArgs& a, const Work& w, i
 // reference max while the scores stream in from TMEM chunk by chunk; only if
 // some row of the warp finds a max more than 8 above its reference (always on
 // the first tile) is the tile redone against the new max, with O rescaled.
-template <int D, bool DECODE, int MOD>
+template <int D, bool DECODE, int MOD, bool BM>
 __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, int s, int row, int t, int cls,
                                              uint32_t tS, uint32_t tO, bool first, RowState& st,
                                              uint64_t* p_ready) {
@@ -684,9 +688,9 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
     float guess_ref = NEG_INF;
     const float my_nmu = my_guess ? 0.0f : -st.m;
     if (cls == 2)
-      mt = stream_tile<DECODE, MOD, false>(a, w, s, row, t, tS, x, my_nmu, acc0, acc1, my_guess, guess_ref) * mult;
+      mt = stream_tile<DECODE, MOD, false, BM>(a, w, s, row, t, tS, x, my_nmu, acc0, acc1, my_guess, guess_ref) * mult;
     else
-      mt = stream_tile<DECODE, MOD, true>(a, w, s, row, t, tS, x, my_nmu, acc0, acc1, my_guess, guess_ref) * mult;
+      mt = stream_tile<DECODE, MOD, true, BM>(a, w, s, row, t, tS, x, my_nmu, acc0, acc1, my_guess, guess_ref) * mult;
     if (my_guess) {
       // This row's exponentials are relative to the guess, which becomes its
       // reference; its l and O are still empty (or all zero).
@@ -699,9 +703,9 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
     // reference max when there is one, else in the slow path below.
     float mc;
     if (cls == 2)
-      mc = prepare_tile<DECODE, MOD, false>(a, w, s, row, t, tS, x);
+      mc = prepare_tile<DECODE, MOD, false, BM>(a, w, s, row, t, tS, x);
     else
-      mc = prepare_tile<DECODE, MOD, true>(a, w, s, row, t, tS, x);
+      mc = prepare_tile<DECODE, MOD, true, BM>(a, w, s, row, t, tS, x);
     mt = mc * mult;
     if (have_ref) {
       const float2 NMU = make_float2(nmu0, nmu0);
@@ -886,7 +890,7 @@ __device__ __forceinline__ bool epilogue(const FwdArgs& a, const CUtensorMap* ma
 //   k_full / v_full / kv_empty            once per K/V load.
 // While the softmax warps write a unit's outputs, the producer already loads
 // the next unit's Q and K/V and the MMA warp runs its first QK^T products.
-template <int D, bool DECODE, int MOD>
+template <int D, bool DECODE, int MOD, bool BM>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
@@ -958,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (u < 0) continue;
       const Work w = map_work<DECODE>(a, u);
       TileWalker tw;
-      const int n = walker_init<DECODE>(a, w, tw);
+      const int n = walker_init<DECODE, BM>(a, w, tw);
       if (n == 0) continue;
       if (qcnt > 0 && !wait_all(&bar.q_empty, (qcnt - 1) & 1)) {
         ok = false;
@@ -996,7 +1000,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (DECODE)
           ++tw.t;
         else
-          walker_next(a, tw);
+          walker_next<BM>(tw);
       }
     }
     // Drain: on an abort, wait (bounded) for every copy still in flight so
@@ -1039,25 +1043,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto slot_of = [&](int g, int s) { return DECODE ? (2 * g + s) % L::kNSlot : g % L::kNSlot; };
     auto phase_of = [&](int g, int s) { return (uint32_t)(((DECODE ? 2 * g + s : g) / L::kNSlot) & 1); };
+    // Steps of round r's unit (0 if it has none). The MMA warp needs nothing
+    // else about a unit. The next round's count is taken right after a
+    // unit's first QK^T products are issued, while the softmax works on
+    // them: this once-per-unit code has usually left the instruction cache,
+    // and its refetch is hidden there instead of delaying the next QK^T.
+    auto unit_steps = [&](int r) -> int {
+      const int u = r < rounds ? unit_of(r) : -1;
+      if (u < 0) return 0;
+      const Work w = map_work<DECODE>(a, u);
+      TileWalker tw;
+      return walker_init<DECODE, BM>(a, w, tw);
+    };
     int gstep = 0;  // steps issued so far across units
     int qcnt = 0;   // units with key tiles so far
     bool ok = true;
+    int n_next = unit_steps(0);
     for (int r = 0; ok && r < rounds; ++r) {
-      const int u = unit_of(r);
-      if (u < 0) continue;
-      const Work w = map_work<DECODE>(a, u);
-      TileWalker tw;
-      const int n = walker_init<DECODE>(a, w, tw);
-      if (n == 0) continue;
-      ok = wait_all(&bar.q_full, qcnt & 1);
-      if (ok) ok = wait_all(&bar.k_full[slot_of(gstep, 0)], phase_of(gstep, 0));
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0, slot_of(gstep, 0), false);
-        if (DECODE) ok = wait_all(&bar.k_full[slot_of(gstep, 1)], phase_of(gstep, 1));
-        tc_fence_after();
-        if (ok) issue_qk(1, slot_of(gstep, 1), n == 1);
+      const int n = n_next;
+      if (n > 0) {
+        ok = wait_all(&bar.q_full, qcnt & 1);
+        if (ok) ok = wait_all(&bar.k_full[slot_of(gstep, 0)], phase_of(gstep, 0));
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, slot_of(gstep, 0), false);
+          if (DECODE) ok = wait_all(&bar.k_full[slot_of(gstep, 1)], phase_of(gstep, 1));
+          tc_fence_after();
+          if (ok) issue_qk(1, slot_of(gstep, 1), n == 1);
+        }
       }
+      n_next = unit_steps(r + 1);
+      if (n == 0) continue;
       for (int j = 0; ok && j < n; ++j) {
         const int g = gstep + j;
         const bool more = j + 1 < n;
@@ -1106,37 +1122,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = lane_base + 256 + s * L::kOCols;
     int gstep = 0, qcnt = 0;
     bool ok = true;
+    // The next round's unit is set up while this warp waits for the current
+    // unit's last PV (once-per-unit code, usually refetched into the
+    // instruction cache), not after the epilogue.
+    int u_next;
+    Work w_next;
+    TileWalker tw_next;
+    int n_next = 0;
+    auto setup = [&](int r) {
+      u_next = r < rounds ? unit_of(r) : -1;
+      if (u_next >= 0) {
+        w_next = map_work<DECODE>(a, u_next);
+        n_next = walker_init<DECODE, BM>(a, w_next, tw_next);
+      }
+    };
+    setup(0);
     for (int r = 0; ok && r < rounds; ++r) {
-      const int u = unit_of(r);
-      if (u < 0) continue;
-      const Work w = map_work<DECODE>(a, u);
-      TileWalker tw;
-      const int n = walker_init<DECODE>(a, w, tw);
+      const bool have_unit = u_next >= 0;
+      const Work w = w_next;
+      TileWalker tw = tw_next;
+      const int n = have_unit ? n_next : 0;
       RowState st;
       st.m = -__int_as_float(0x7f800000);
       st.l = 0.f;
-      if (n == 0) {
-        epilogue<D, DECODE>(a, &map_o, w, s, row, lane_base, false, st, extra, bar, qcnt, abort_flag);
-        continue;
-      }
       if (DECODE) tw.t += s;
       for (int j = 0; j < n; ++j) {
         const int t = tw.t;
-        const int cls = tile_class<DECODE>(a, w, s, t);
+        const int cls = tile_class<DECODE, BM>(a, w, s, t);
         if (!wait_all(&bar.s_ready[s], (gstep + j) & 1)) { ok = false; break; }
         tc_fence_after();
-        softmax_step<D, DECODE, MOD>(a, w, s, row, t, cls, tS, tO, j == 0, st, &bar.p_ready[s]);
+        softmax_step<D, DECODE, MOD, BM>(a, w, s, row, t, cls, tS, tO, j == 0, st, &bar.p_ready[s]);
         if (DECODE)
           tw.t += 2;
         else
-          walker_next(a, tw);
+          walker_next<BM>(tw);
       }
       if (!ok) break;
-      bool got = wait_all(&bar.o_done[s], qcnt & 1);
-      if (DECODE && s == 0) got = got && wait_all(&bar.o_done[1], qcnt & 1);
-      if (!got) break;
-      tc_fence_after();
-      if (!epilogue<D, DECODE>(a, &map_o, w, s, row, lane_base, true, st, extra, bar, qcnt, abort_flag)) break;
+      setup(r + 1);
+      if (!have_unit) continue;
+      if (n > 0) {
+        bool got = wait_all(&bar.o_done[s], qcnt & 1);
+        if (DECODE && s == 0) got = got && wait_all(&bar.o_done[1], qcnt & 1);
+        if (!got) break;
+        tc_fence_after();
+      }
+      // A unit without key tiles still writes its (all-masked) outputs.
+      if (!epilogue<D, DECODE>(a, &map_o, w, s, row, lane_base, n > 0, st, extra, bar, qcnt, abort_flag)) break;
+      if (n == 0) continue;
       // O is read: the next unit's first PV may overwrite it. In decode the
       // subtile-0 threads read both accumulators and release both.
       tc_fence_before();
