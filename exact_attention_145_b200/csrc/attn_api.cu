@@ -236,8 +236,13 @@ attn_status attn_build_block_mask(const attn_mask_spec* spec, const attn_block_m
   a.full_cnt = out->full_cnt;
   a.full_idx = out->full_idx;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t smem = a.kind == ATTN_MASK_DOCUMENT ? (size_t)kKvPerCta * a.blk_kv * sizeof(int) : 0;
-  classify_tiles_kernel<<<dim3(a.nQ, (a.nK + kKvPerCta - 1) / kKvPerCta), kMaskThreads, smem, st>>>(a);
+  if (a.kind == ATTN_MASK_DOCUMENT) {
+    const size_t smem = (size_t)kKvPerCta * a.blk_kv * sizeof(int);
+    classify_doc_kernel<<<dim3(a.nQ, (a.nK + kKvPerCta - 1) / kKvPerCta), kMaskThreads, smem, st>>>(a);
+  } else {
+    const int64_t tiles = (int64_t)a.nQ * a.nK;
+    classify_range_kernel<<<(unsigned)((tiles + 255) / 256), 256, 0, st>>>(a);
+  }
   compact_lists_kernel<<<a.nQ, 32, 0, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -16,57 +16,130 @@ struct MaskArgs {
   int32_t *part_cnt, *part_idx, *full_cnt, *full_idx;
 };
 
-// Block-mask build, pass 1: classify tiles. CTA (q-tile, group of kKvPerCta
-// kv-tiles); each thread evaluates its query rows against every in-range key
-// of a tile (stopping early once it has seen both an allowed and a masked
-// pair), then block votes give "any allowed" and "all allowed".
+// Block-mask build, pass 1: classify tiles (0 empty, 1 partial, 2 full).
+// Only in-range positions of ragged edge tiles count.
 constexpr int kMaskThreads = 128;
 constexpr int kKvPerCta = 8;
 
-__device__ __forceinline__ bool pair_allowed(const MaskArgs& a, long q_pos, int j, int doc_i, int doc_j) {
-  switch (a.kind) {
-    case 0:
-      return true;
-    case 1:
-      return (long)j <= q_pos;
-    case 2:
-      return (a.wl < 0 || q_pos - j <= a.wl) && (a.wr < 0 || (long)j - q_pos <= a.wr);
-    default:
-      return (long)j <= q_pos && doc_j == doc_i;
+// Window forms (none, causal, window): one thread per tile, exact interval
+// arithmetic. The keys a query at position p may see form the window
+// [p - wl, p + wr] (a side with a negative bound is unbounded). Over a tile's
+// rows q0..q1 these windows overlap or touch, so their union is the single
+// interval [q0 - wl, q1 + wr]: the tile is empty iff its keys k0..k1 miss that
+// interval, and full iff every key lies in every row's window,
+// i.e. k0 >= q1 - wl and k1 <= q0 + wr.
+__global__ void __launch_bounds__(256) classify_range_kernel(const MaskArgs a) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)a.nQ * a.nK) return;
+  const int qt = (int)(i / a.nK), kt = (int)(i % a.nK);
+  const long q0 = (long)qt * a.blk_q + a.q_offset;
+  const long q1 = (long)min((qt + 1) * a.blk_q, a.Sq) - 1 + a.q_offset;
+  const long k0 = (long)kt * a.blk_kv;
+  const long k1 = (long)min((kt + 1) * a.blk_kv, a.Skv) - 1;
+  bool empty = false, full = true;
+  if (a.kind != 0) {
+    if (a.wl >= 0) {
+      if (k1 < q0 - a.wl) empty = true;
+      if (k0 < q1 - a.wl) full = false;
+    }
+    if (a.wr >= 0) {
+      if (k0 > q1 + a.wr) empty = true;
+      if (k1 > q0 + a.wr) full = false;
+    }
+  }
+  a.cls[i] = empty ? 0 : (full ? 2 : 1);
+}
+
+__device__ __forceinline__ void warp_minmax(int& lo, int& hi) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
   }
 }
 
-__global__ void __launch_bounds__(kMaskThreads) classify_tiles_kernel(const MaskArgs a) {
-  extern __shared__ int doc_k[];  // [kKvPerCta * blk_kv] key doc ids (document masks)
+// Document mask (key j visible to query i iff doc[j] == doc[i] and j <= i):
+// one CTA per (q-tile, kKvPerCta kv-tiles). The id ranges of the two sides
+// decide most tiles at once: keys all past the last query -> empty; disjoint
+// id ranges -> empty; one id shared by every position of both tiles -> the
+// causal class. The remaining tiles (those crossing a document boundary, or
+// any tile when the ids are not grouped) are evaluated pair by pair: each
+// thread walks its query rows against the tile's keys, stopping once it has
+// seen both an allowed and a masked pair, and block votes give "any" and "all".
+__global__ void __launch_bounds__(kMaskThreads) classify_doc_kernel(const MaskArgs a) {
+  extern __shared__ int doc_k[];  // [kKvPerCta * blk_kv] key doc ids
+  __shared__ int red_lo[kMaskThreads / 32], red_hi[kMaskThreads / 32];
+  __shared__ int tile_lo[kKvPerCta], tile_hi[kKvPerCta];
   const int qt = blockIdx.x;
   const int kt0 = blockIdx.y * kKvPerCta;
   const int kt1 = min(kt0 + kKvPerCta, a.nK);
   const int q0 = qt * a.blk_q;
   const int rows = min(a.blk_q, a.Sq - q0);
-  const bool is_doc = a.kind == 3;
-  if (is_doc) {
-    const int k_first = kt0 * a.blk_kv, k_end = min(kt1 * a.blk_kv, a.Skv);
-    for (int c = threadIdx.x; c < k_end - k_first; c += blockDim.x) doc_k[c] = a.doc_id[k_first + c];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int k_first = kt0 * a.blk_kv, k_end = min(kt1 * a.blk_kv, a.Skv);
+  for (int c = threadIdx.x; c < k_end - k_first; c += blockDim.x) doc_k[c] = a.doc_id[k_first + c];
+  // id range of the query tile
+  int lo = 0x7fffffff, hi = -0x7fffffff - 1;
+  for (int r = threadIdx.x; r < rows; r += blockDim.x) {
+    const int d = a.doc_id[q0 + r];
+    lo = min(lo, d);
+    hi = max(hi, d);
+  }
+  warp_minmax(lo, hi);
+  if (lane == 0) {
+    red_lo[warp] = lo;
+    red_hi[warp] = hi;
+  }
+  __syncthreads();
+  int qlo = red_lo[0], qhi = red_hi[0];
+#pragma unroll
+  for (int w = 1; w < kMaskThreads / 32; ++w) {
+    qlo = min(qlo, red_lo[w]);
+    qhi = max(qhi, red_hi[w]);
+  }
+  // id range of each key tile, one warp per tile
+  for (int kt = kt0 + warp; kt < kt1; kt += kMaskThreads / 32) {
+    const int base = (kt - kt0) * a.blk_kv;
+    const int cols = min(a.blk_kv, a.Skv - kt * a.blk_kv);
+    int l2 = 0x7fffffff, h2 = -0x7fffffff - 1;
+    for (int c = lane; c < cols; c += 32) {
+      l2 = min(l2, doc_k[base + c]);
+      h2 = max(h2, doc_k[base + c]);
+    }
+    warp_minmax(l2, h2);
+    if (lane == 0) {
+      tile_lo[kt - kt0] = l2;
+      tile_hi[kt - kt0] = h2;
+    }
   }
   __syncthreads();
   for (int kt = kt0; kt < kt1; ++kt) {
     const int k0 = kt * a.blk_kv;
     const int cols = min(a.blk_kv, a.Skv - k0);
-    const int* dk = doc_k + (kt - kt0) * a.blk_kv;
-    bool any = false, all = true;
-    for (int r = threadIdx.x; r < rows && (all || !any); r += blockDim.x) {
-      const long q_pos = (long)(q0 + r) + a.q_offset;
-      const int di = is_doc ? a.doc_id[q0 + r] : 0;
-      for (int c = 0; c < cols; ++c) {
-        const bool ok = pair_allowed(a, q_pos, k0 + c, di, is_doc ? dk[c] : 0);
-        any |= ok;
-        all &= ok;
-        if (any && !all) break;
+    const int klo = tile_lo[kt - kt0], khi = tile_hi[kt - kt0];
+    int cls;
+    if (k0 > q0 + rows - 1 || khi < qlo || klo > qhi) {
+      cls = 0;
+    } else if (qlo == qhi && klo == khi && qlo == klo) {
+      cls = (k0 + cols - 1 <= q0) ? 2 : 1;
+    } else {
+      const int* dk = doc_k + (kt - kt0) * a.blk_kv;
+      bool any = false, all = true;
+      for (int r = threadIdx.x; r < rows && (all || !any); r += blockDim.x) {
+        const int qi = q0 + r;
+        const int di = a.doc_id[qi];
+        for (int c = 0; c < cols; ++c) {
+          const bool ok = k0 + c <= qi && dk[c] == di;
+          any |= ok;
+          all &= ok;
+          if (any && !all) break;
+        }
       }
+      const int any_b = __syncthreads_or(any);
+      const int all_b = __syncthreads_and(all);
+      cls = any_b ? (all_b ? 2 : 1) : 0;
     }
-    const int any_b = __syncthreads_or(any);
-    const int all_b = __syncthreads_and(all);
-    if (threadIdx.x == 0) a.cls[(int64_t)qt * a.nK + kt] = any_b ? (all_b ? 2 : 1) : 0;
+    if (threadIdx.x == 0) a.cls[(int64_t)qt * a.nK + kt] = (uint8_t)cls;
   }
 }
 

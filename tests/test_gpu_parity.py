@@ -177,6 +177,36 @@ def test_block_mask_ragged_exact(Sq, Skv, blk):
         _bm_compare(bm, ref)
 
 
+@pytest.mark.parametrize("S,blk,ids", [(1000, 64, "sorted"), (777, 16, "unsorted"), (1500, 128, "unsorted"),
+                                       (2048, 128, "two"), (300, 128, "one")])
+def test_block_mask_document_exact(S, blk, ids):
+    """Document classes: tiles decided from id ranges (sorted, one or two
+    documents) and tiles evaluated pair by pair (unsorted ids mix every tile)."""
+    if ids == "sorted":
+        doc = W.doc_ids_from_lengths(W.doc_lengths(99, S, 20, 300))
+    elif ids == "unsorted":
+        doc = W.uniform_ints(123 + S, S, 0, 3)
+    elif ids == "two":
+        doc = np.zeros(S, np.int32)
+        doc[S // 3:] = 1
+    else:
+        doc = np.full(S, 7, np.int32)
+    ref = oracle.block_mask(W.MASK_DOCUMENT, S, S, blk, blk, doc_id=doc)
+    bm = ea.attn_build_block_mask(S, S, doc_id=torch.from_numpy(doc).cuda(), blk_q=blk, blk_kv=blk)
+    torch.cuda.synchronize()
+    _bm_compare(bm, ref)
+
+
+@pytest.mark.parametrize("window,q_off", [((0, 0), 0), ((0, 0), -5), ((3, 40), 200), ((-1, 5), -300), ((200, -1), 0)])
+def test_block_mask_window_edges_exact(window, q_off):
+    """Interval classification at narrow bands, offsets that push rows off the key range, one-sided windows."""
+    for Sq, Skv, blk in [(500, 700, 64), (129, 128, 16), (1024, 1024, 128)]:
+        ref = oracle.block_mask(W.MASK_WINDOW, Sq, Skv, blk, blk, window=window, q_offset=q_off)
+        bm = ea.attn_build_block_mask(Sq, Skv, window=window, q_offset=q_off, blk_q=blk, blk_kv=blk)
+        torch.cuda.synchronize()
+        _bm_compare(bm, ref)
+
+
 def test_block_mask_drives_causal_like_analytic():
     S = 900
     q = W.normal_bf16(101, (1, S, 4, 128))

@@ -103,6 +103,11 @@ def doc_ids_from_lengths(lens) -> np.ndarray:
     return np.repeat(np.arange(len(lens), dtype=np.int32), lens)
 
 
+def uniform_ints(seed: int, n: int, lo: int, hi: int) -> np.ndarray:
+    """n int32 values uniform in [lo, hi] (splitmix64 modulo the span)."""
+    return (lo + splitmix64(seed, n) % np.uint64(hi - lo + 1)).astype(np.int32)
+
+
 def page_permutation(seed: int, num_pages: int) -> np.ndarray:
     """Fisher-Yates shuffle of range(num_pages) driven by splitmix64(seed)."""
     perm = np.arange(num_pages, dtype=np.int32)
