@@ -123,16 +123,25 @@ __global__ void __launch_bounds__(kMaskThreads) classify_doc_kernel(const MaskAr
     } else if (qlo == qhi && klo == khi && qlo == klo) {
       cls = (k0 + cols - 1 <= q0) ? 2 : 1;
     } else {
-      const int* dk = doc_k + (kt - kt0) * a.blk_kv;
+      // Eight keys per iteration from two 16-byte shared loads (blk_kv is a
+      // multiple of 16, so every group starts 32-byte aligned); keys past
+      // the ragged end of the sequence are skipped.
+      const int4* dk4 = reinterpret_cast<const int4*>(doc_k + (kt - kt0) * a.blk_kv);
       bool any = false, all = true;
       for (int r = threadIdx.x; r < rows && (all || !any); r += blockDim.x) {
         const int qi = q0 + r;
         const int di = a.doc_id[qi];
-        for (int c = 0; c < cols; ++c) {
-          const bool ok = k0 + c <= qi && dk[c] == di;
-          any |= ok;
-          all &= ok;
-          if (any && !all) break;
+        for (int c = 0; c < cols && (all || !any); c += 8) {
+          const int4 d0 = dk4[c / 4], d1 = dk4[c / 4 + 1];
+          const int dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (c + e < cols) {
+              const bool ok = k0 + c + e <= qi && dd[e] == di;
+              any |= ok;
+              all &= ok;
+            }
+          }
         }
       }
       const int any_b = __syncthreads_or(any);

@@ -944,6 +944,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool got = mbar_wait(b, par, abort_flag);
     return __all_sync(0xffffffffu, got);
   };
+  // Polling variant for the per-step S-ready / P-ready hand-offs.
+  auto wait_spin_all = [&](uint64_t* b, uint32_t par) {
+    const bool got = mbar_wait_spin(b, par, abort_flag);
+    return __all_sync(0xffffffffu, got);
+  };
 
   if (warp == kTmaWarp) {
     regs_decrease<kControlRegs>();
@@ -1081,7 +1086,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s) {
           const int slot = slot_of(g, s);
           if (!wait_all(&bar.v_full[slot], phase_of(g, s))) { ok = false; break; }
-          if (!wait_all(&bar.p_ready[s], g & 1)) { ok = false; break; }
+          if (!wait_spin_all(&bar.p_ready[s], g & 1)) { ok = false; break; }
           // The first PV of a unit overwrites O(s): the previous unit's epilogue must have read it.
           if (j == 0 && qcnt > 0 && !wait_all(&bar.o_free[s], (qcnt - 1) & 1)) { ok = false; break; }
           tc_fence_after();
@@ -1149,7 +1154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j) {
         const int t = tw.t;
         const int cls = tile_class<DECODE, BM>(a, w, s, t);
-        if (!wait_all(&bar.s_ready[s], (gstep + j) & 1)) { ok = false; break; }
+        if (!wait_spin_all(&bar.s_ready[s], (gstep + j) & 1)) { ok = false; break; }
         tc_fence_after();
         softmax_step<D, DECODE, MOD, BM>(a, w, s, row, t, cls, tS, tO, j == 0, st, &bar.p_ready[s]);
         if (DECODE)

@@ -88,6 +88,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// The same bounded wait without the suspend hint: the thread polls, so it
+// resumes as soon as the phase completes instead of after the hardware wake-up.
+// Used for the per-key-tile hand-offs on the critical path (S ready, P ready),
+// where the wake-up latency sits between the softmax and the tensor pipe.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const long long t0 = clock64();
+  while (!mbar_test(bar, parity)) {
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitTimeoutCycles) {
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
 // Same wait without an abort flag, for teardown: gives up after the timeout.
 __device__ __forceinline__ bool mbar_wait_timeout(uint64_t* bar, uint32_t parity) {
   if (mbar_test(bar, parity)) return true;
