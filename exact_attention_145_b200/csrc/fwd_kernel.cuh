@@ -516,9 +516,13 @@ __device__ __forceinline__ MaskRow mask_row(const FwdArgs& a, const Work& w, int
 // the prefill window forms (causal included) the row's allowed range becomes
 // a 32-bit mask for the chunk, so each element costs one bit test and one
 // select; decode (only a split's ragged last tile) and the document mask keep
-// the range compare, which needs fewer live registers.
+// the range compare, which needs fewer live registers. Without a block mask
+// (BM false) a chunk allowed for the whole warp skips the selects, and the
+// return value tells the caller that a chunk is masked for every row of the
+// warp, so its exponentials are skipped (in block-mask kernels these votes
+// cost more registers than they save).
 template <bool DECODE, bool BM>
-__device__ __forceinline__ void mask_chunk(const FwdArgs& a, const MaskRow& m, int t, int c, float* x) {
+__device__ __forceinline__ bool mask_chunk(const FwdArgs& a, const MaskRow& m, int t, int c, float* x) {
   const float NEG_INF = -__int_as_float(0x7f800000);
   if (BM && a.mask == MASK_DOCUMENT) {
     const int kv = t * kKeys + 32 * c;
@@ -539,15 +543,20 @@ __device__ __forceinline__ void mask_chunk(const FwdArgs& a, const MaskRow& m, i
       x[4 * i4 + 2] = (!m.none && (unsigned)(j + 2 - m.clo) <= m.span && d.z == m.dq) ? x[4 * i4 + 2] : NEG_INF;
       x[4 * i4 + 3] = (!m.none && (unsigned)(j + 3 - m.clo) <= m.span && d.w == m.dq) ? x[4 * i4 + 3] : NEG_INF;
     }
+    return false;
   } else if constexpr (DECODE) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) x[i] = (!m.none && (unsigned)(32 * c + i - m.clo) <= m.span) ? x[i] : NEG_INF;
+    return false;
   } else {
     const int lo = m.clo - 32 * c, hi = m.clo + (int)m.span - 32 * c;
     unsigned bits = 0u;
     if (!m.none && hi >= 0 && lo <= 31) bits = (0xffffffffu >> (31 - min(hi, 31))) & (0xffffffffu << max(lo, 0));
+    if (!BM && __all_sync(0xffffffffu, bits == 0xffffffffu)) return false;
+    const bool dead = !BM && __all_sync(0xffffffffu, bits == 0u);
 #pragma unroll
     for (int i = 0; i < 32; ++i) x[i] = (bits & (1u << i)) ? x[i] : NEG_INF;
+    return dead;
   }
 }
 
@@ -605,7 +614,8 @@ __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, in
   for (int c = 0; c < 4; ++c) {
     if (c < 3) tmem_ld32f(tS + 32 * (c + 1), x + 32 * (c + 1));
     if constexpr (MOD != MOD_NONE) mod_chunk<DECODE, MOD>(a, w, s, row, t, c, x + 32 * c);
-    if constexpr (MASKED) mask_chunk<DECODE, BM>(a, mr, t, c, x + 32 * c);
+    bool dead = false;
+    if constexpr (MASKED) dead = mask_chunk<DECODE, BM>(a, mr, t, c, x + 32 * c);
     mc = fmaxf(mc, chunk_max(x + 32 * c));
     if (c == 0 && guess) {
       const float g = mc * mult;
@@ -613,7 +623,13 @@ __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, in
       NMU = make_float2(g == NEG_INF ? 0.0f : -g, g == NEG_INF ? 0.0f : -g);
     }
     uint32_t pk[16];
-    exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
+    if (MASKED && !BM && dead) {
+      // every score of this chunk is masked for the whole warp: P = 0
+#pragma unroll
+      for (int j = 0; j < 16; ++j) pk[j] = 0u;
+    } else {
+      exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
+    }
     tmem_st16(tS + 16 * c, pk);
     if (c < 3) {
       tmem_ld_wait();
@@ -640,7 +656,7 @@ __device__ __forceinline__ float prepare_tile(const FwdArgs& a, const Work& w, i
   for (int c = 0; c < 4; ++c) {
     if (c < 3) tmem_ld32f(tS + 32 * (c + 1), x + 32 * (c + 1));
     if constexpr (MOD != MOD_NONE) mod_chunk<DECODE, MOD>(a, w, s, row, t, c, x + 32 * c);
-    if constexpr (MASKED) mask_chunk<DECODE, BM>(a, mr, t, c, x + 32 * c);
+    if constexpr (MASKED) (void)mask_chunk<DECODE, BM>(a, mr, t, c, x + 32 * c);
     mc = fmaxf(mc, chunk_max(x + 32 * c));
     if (c < 3) {
       tmem_ld_wait();
