@@ -123,8 +123,11 @@ struct Barriers {
   uint64_t k_full[6];
   uint64_t v_full[6];
   uint64_t kv_empty[6];
-  uint64_t s_ready[2];
-  uint64_t p_ready[2];
+  uint64_t s_ready[2];    // prefill: keys 0-63 of S ready (decode: the whole S)
+  uint64_t p_ready[2];    // prefill: P for keys 0-63 written (decode: the whole P)
+  uint64_t s_b_ready[2];  // prefill: keys 64-127 of S ready
+  uint64_t p_b_ready[2];  // prefill: P for keys 64-127 written
+  uint64_t pv_a_done[2];  // prefill: the PV of keys 0-63 has completed
   uint64_t o_done[2];
   uint64_t o_free[2];
   uint64_t merge_full, merge_empty;  // decode: subtile-1 row stats handed to subtile 0
@@ -778,6 +781,232 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
   st.l = st.l * alpha + (acc0.x + acc0.y);
 }
 
+// ---------------------------------------------------------------- prefill, half tiles
+// Kernels with a score mod (softcap, ALiBi) hand each key tile to the tensor
+// pipe in two halves; their softmax is long enough that overlapping it with
+// the MMAs pays for the extra hand-offs (+6-8 % measured). Without a mod the
+// whole-tile schedule is faster (the half schedule measured 5 % slower).
+template <bool DECODE, int MOD>
+constexpr bool kHalfTiles = !DECODE && MOD != MOD_NONE;
+
+// With half tiles: P for keys
+// 0-63 goes to S(s) columns [0, 32) and P for keys 64-127 to [64, 96), so:
+//   - once P of keys 0-63 is written, PV over those keys and the next tile's
+//     QK^T for keys 0-63 (into columns [0, 64)) run while the softmax works on
+//     keys 64-127;
+//   - once P of keys 64-127 is written, PV over them and the next tile's
+//     QK^T for keys 64-127 (into [64, 128)) follow.
+// The softmax of the next tile starts on its first half while the tensor
+// pipe finishes the second, so neither waits for the other's whole tile.
+
+// Half h of a key tile (chunks 2h, 2h+1: S(s) columns [64h, 64h+64)),
+// streamed like stream_tile: chunk 2h+1 is in flight while chunk 2h is
+// exponentiated. x holds the half's 64 scores.
+template <int MOD, bool MASKED, bool BM>
+__device__ __forceinline__ float stream_half(const FwdArgs& a, const Work& w, int s, int row, int t, uint32_t tS,
+                                             int h, float* x, float nmu0, float2& acc0, float2& acc1, bool guess,
+                                             float& ref_out) {
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  const float mult = MOD == MOD_NONE ? a.scale_log2 : 1.0f;
+  const float2 MULT = make_float2(mult, mult);
+  float2 NMU = make_float2(nmu0, nmu0);
+  MaskRow mr;
+  if constexpr (MASKED) mr = mask_row<false, BM>(a, w, s, row, t);
+  float mc = NEG_INF;
+  const uint32_t base = tS + 64 * h;
+  tmem_ld32f(base, x);
+  tmem_ld_wait();
+  reg_fence_f<32>(x);
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    const int c = 2 * h + cc;
+    if (cc == 0) tmem_ld32f(base + 32, x + 32);
+    if constexpr (MOD != MOD_NONE) mod_chunk<false, MOD>(a, w, s, row, t, c, x + 32 * cc);
+    bool dead = false;
+    if constexpr (MASKED) dead = mask_chunk<false, BM>(a, mr, t, c, x + 32 * cc);
+    mc = fmaxf(mc, chunk_max(x + 32 * cc));
+    if (cc == 0 && guess) {
+      const float g = mc * mult;
+      ref_out = g;
+      NMU = make_float2(g == NEG_INF ? 0.0f : -g, g == NEG_INF ? 0.0f : -g);
+    }
+    uint32_t pk[16];
+    if (MASKED && !BM && dead) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) pk[j] = 0u;
+    } else {
+      exp_chunk(x + 32 * cc, MULT, NMU, pk, acc0, acc1);
+    }
+    tmem_st16(base + 16 * cc, pk);
+    if (cc == 0) {
+      tmem_ld_wait();
+      reg_fence_f<32>(x + 32);
+    }
+  }
+  return mc;
+}
+
+// Half h with score mods: the half's scores (mods, mask) first, then its
+// exponentials once the reference is known.
+template <int MOD, bool MASKED, bool BM>
+__device__ __forceinline__ float prepare_half(const FwdArgs& a, const Work& w, int s, int row, int t, uint32_t tS,
+                                              int h, float* x) {
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  MaskRow mr;
+  if constexpr (MASKED) mr = mask_row<false, BM>(a, w, s, row, t);
+  float mc = NEG_INF;
+  const uint32_t base = tS + 64 * h;
+  tmem_ld32f(base, x);
+  tmem_ld_wait();
+  reg_fence_f<32>(x);
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    const int c = 2 * h + cc;
+    if (cc == 0) tmem_ld32f(base + 32, x + 32);
+    if constexpr (MOD != MOD_NONE) mod_chunk<false, MOD>(a, w, s, row, t, c, x + 32 * cc);
+    if constexpr (MASKED) (void)mask_chunk<false, BM>(a, mr, t, c, x + 32 * cc);
+    mc = fmaxf(mc, chunk_max(x + 32 * cc));
+    if (cc == 0) {
+      tmem_ld_wait();
+      reg_fence_f<32>(x + 32);
+    }
+  }
+  return mc;
+}
+
+// Multiplies this row's O accumulator by alpha in TMEM.
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < D; c += 32) {
+    float o[32];
+    tmem_ld32f(tO + c, o);
+    tmem_ld_wait();
+    reg_fence_f<32>(o);
+    uint32_t ob[32];
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const float2 r = mul2(make_float2(o[j], o[j + 1]), make_float2(alpha, alpha));
+      ob[j] = __float_as_uint(r.x);
+      ob[j + 1] = __float_as_uint(r.y);
+    }
+    tmem_st32(tO + c, ob);
+  }
+}
+
+// One key tile of the prefill online softmax for one query row, as two
+// halves. The exponentials of a half are taken against the row's reference
+// max (the first chunk's max when the row has none yet); when some row of
+// the warp finds the half's max more than 8 above its reference, the half is
+// redone against the new max and O is rescaled, after waiting for the PVs
+// that may still be adding into O: for the first half, the previous tile's
+// second-half PV (done once this tile's keys 64-127 are in S); for the second
+// half, this tile's first-half PV. On entry S of keys 0-63 is ready. g is the
+// step's barrier phase index; returns false if a wait gave up.
+template <int D, int MOD, bool BM>
+__device__ __forceinline__ bool softmax_step_halves(const FwdArgs& a, const Work& w, int s, int row, int t, int cls,
+                                                    uint32_t tS, uint32_t tO, bool first, RowState& st, Barriers& bar,
+                                                    int g, volatile int* abort_flag) {
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  const float mult = MOD == MOD_NONE ? a.scale_log2 : 1.0f;
+  const float2 MULT = make_float2(mult, mult);
+  const uint32_t par = (uint32_t)(g & 1);
+  bool b_ready = false;  // S of keys 64-127 already waited for
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    if (h == 1 && !b_ready) {
+      if (!__all_sync(0xffffffffu, mbar_wait_spin(&bar.s_b_ready[s], par, abort_flag))) return false;
+      tc_fence_after();
+    }
+    float x[64];
+    float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+    float mh;
+    const bool have_ref = __all_sync(0xffffffffu, st.m != NEG_INF);
+    bool guessed = false;
+    if (cls == 0) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c) x[c] = NEG_INF;
+      mh = NEG_INF;
+      uint32_t pk[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) pk[j] = 0u;
+      tmem_st32(tS + 64 * h, pk);
+      guessed = true;
+    } else if (MOD == MOD_NONE) {
+      const bool my_guess = st.m == NEG_INF;
+      float guess_ref = NEG_INF;
+      const float my_nmu = my_guess ? 0.0f : -st.m;
+      if (cls == 2)
+        mh = stream_half<MOD, false, BM>(a, w, s, row, t, tS, h, x, my_nmu, acc0, acc1, my_guess, guess_ref) * mult;
+      else
+        mh = stream_half<MOD, true, BM>(a, w, s, row, t, tS, h, x, my_nmu, acc0, acc1, my_guess, guess_ref) * mult;
+      if (my_guess) {
+        // the guess becomes this row's reference; its l and O hold nothing yet
+        st.m = guess_ref;
+        st.l = 0.0f;
+      }
+      guessed = true;
+    } else {
+      float mc;
+      if (cls == 2)
+        mc = prepare_half<MOD, false, BM>(a, w, s, row, t, tS, h, x);
+      else
+        mc = prepare_half<MOD, true, BM>(a, w, s, row, t, tS, h, x);
+      mh = mc * mult;
+      if (have_ref) {
+        const float2 NMU = make_float2(-st.m, -st.m);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
+          exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
+          tmem_st16(tS + 64 * h + 16 * c, pk);
+        }
+      }
+    }
+    const bool grow = (!have_ref && !guessed) || mh > st.m + kRescaleThreshold;
+    float alpha = 1.0f;
+    if (__any_sync(0xffffffffu, grow) && cls != 0) {
+      const float m_new = fmaxf(st.m, mh);
+      alpha = (m_new == NEG_INF || st.m == NEG_INF) ? (st.m == NEG_INF ? 0.0f : 1.0f) : ex2(st.m - m_new);
+      st.m = m_new;
+      const float nmu = (m_new == NEG_INF) ? 0.0f : -m_new;
+      const float2 NMU = make_float2(nmu, nmu);
+      acc0 = acc1 = make_float2(0.f, 0.f);
+      tmem_st_wait();  // the optimistic P stores land before they are overwritten
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+        exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
+        tmem_st16(tS + 64 * h + 16 * c, pk);
+      }
+      // O may still receive a PV: wait until it has landed, then rescale.
+      bool have_o = true;
+      if (h == 0) {
+        // The first half's PV of this tile is not issued yet; the previous
+        // tile's second-half PV completed before this tile's keys 64-127
+        // were committed to S. At a unit's first tile O holds nothing.
+        have_o = !first;
+        if (have_o) {
+          if (!__all_sync(0xffffffffu, mbar_wait_spin(&bar.s_b_ready[s], par, abort_flag))) return false;
+          b_ready = true;
+        }
+      } else {
+        if (!__all_sync(0xffffffffu, mbar_wait_spin(&bar.pv_a_done[s], par, abort_flag))) return false;
+      }
+      if (have_o) {
+        tc_fence_after();
+        rescale_o<D>(tO, alpha);
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    mbar_arrive(h == 0 ? &bar.p_ready[s] : &bar.p_b_ready[s]);
+    acc0 = add2(acc0, acc1);
+    st.l = st.l * alpha + (acc0.x + acc0.y);
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- kernel
 // Epilogue of one unit for softmax subtile s: O / l to bf16 (prefill) or the
 // merged, normalised split partial (decode), and the LSE.
@@ -932,6 +1161,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar.s_ready[s], 1);
       mbar_init(&bar.p_ready[s], 128);
+      mbar_init(&bar.s_b_ready[s], 1);
+      mbar_init(&bar.p_b_ready[s], 128);
+      mbar_init(&bar.pv_a_done[s], 1);
       mbar_init(&bar.o_done[s], 1);
       mbar_init(&bar.o_free[s], 128);
     }
@@ -1079,6 +1311,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     int gstep = 0;  // steps issued so far across units
     int qcnt = 0;   // units with key tiles so far
     bool ok = true;
+    // Prefill: QK^T and PV in key halves (see "prefill, half tiles").
+    constexpr uint32_t idesc_qk_half = idesc_bf16_f32(128, 64, 0, 0);
+    constexpr uint32_t kHalfKeyUnits = (64 * 128) >> 4;  // 64 K rows of a 128-byte SW128 box
+    auto issue_qk_half = [&](int s, int slot, int h, uint64_t* done, bool last) {
+      const uint32_t qa = q_lo + (uint32_t)s * kTileUnits;
+      const uint32_t ka = k_lo + (uint32_t)slot * kTileUnits + (uint32_t)h * kHalfKeyUnits;
+      if (elect_one_sync()) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
+          mma_ss(tmem + s * 128 + 64 * h, sdesc_join(qa + off, kHi), sdesc_join(ka + off, kHi), idesc_qk_half,
+                 kk > 0);
+        }
+        mma_commit(done);
+        if (last) mma_commit(&bar.q_empty);
+      }
+      __syncwarp();
+    };
     int n_next = unit_steps(0);
     for (int r = 0; ok && r < rounds; ++r) {
       const int n = n_next;
@@ -1087,14 +1337,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = wait_all(&bar.k_full[slot_of(gstep, 0)], phase_of(gstep, 0));
         if (ok) {
           tc_fence_after();
-          issue_qk(0, slot_of(gstep, 0), false);
-          if (DECODE) ok = wait_all(&bar.k_full[slot_of(gstep, 1)], phase_of(gstep, 1));
-          tc_fence_after();
-          if (ok) issue_qk(1, slot_of(gstep, 1), n == 1);
+          if constexpr (!kHalfTiles<DECODE, MOD>) {
+            issue_qk(0, slot_of(gstep, 0), false);
+            if (DECODE) ok = wait_all(&bar.k_full[slot_of(gstep, 1)], phase_of(gstep, 1));
+            tc_fence_after();
+            if (ok) issue_qk(1, slot_of(gstep, 1), n == 1);
+          } else {
+            const int slot = slot_of(gstep, 0);
+            issue_qk_half(0, slot, 0, &bar.s_ready[0], false);
+            issue_qk_half(1, slot, 0, &bar.s_ready[1], false);
+            issue_qk_half(0, slot, 1, &bar.s_b_ready[0], false);
+            issue_qk_half(1, slot, 1, &bar.s_b_ready[1], n == 1);
+          }
         }
       }
       n_next = unit_steps(r + 1);
       if (n == 0) continue;
+      if constexpr (kHalfTiles<DECODE, MOD>) {
+        for (int j = 0; ok && j < n; ++j) {
+          const int g = gstep + j;
+          const bool more = j + 1 < n;
+          const int slot = slot_of(g, 0);
+          const int nslot = slot_of(g + 1, 0);
+          if (!wait_all(&bar.v_full[slot], phase_of(g, 0))) { ok = false; break; }
+          const uint32_t va = v_lo + (uint32_t)slot * kTileUnits;
+#pragma unroll
+          for (int h = 0; h < 2 && ok; ++h) {
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+              if (!wait_spin_all(h == 0 ? &bar.p_ready[s] : &bar.p_b_ready[s], g & 1)) { ok = false; break; }
+              // The first PV of a unit overwrites O(s): the previous unit's epilogue must have read it.
+              if (j == 0 && h == 0 && qcnt > 0 && !wait_all(&bar.o_free[s], (qcnt - 1) & 1)) { ok = false; break; }
+              tc_fence_after();
+              if (elect_one_sync()) {
+                // PV over keys 64h..64h+63: P from S(s) columns [64h, 64h+32), V rows 64h..
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_ts(tmem + 256 + s * L::kOCols, tmem + s * 128 + 64 * h + kk * 8,
+                         sdesc_join(va + (((4 * h + kk) * 16 * 128) >> 4), kHi), idesc_pv,
+                         (j == 0 && h == 0 && kk == 0) ? 0u : 1u);
+                if (h == 0) mma_commit(&bar.pv_a_done[s]);
+                if (h == 1 && !more) mma_commit(&bar.o_done[s]);
+                if (h == 1 && s == 1) mma_commit(&bar.kv_empty[slot]);
+              }
+              __syncwarp();
+              if (more) {
+                if (h == 0 && s == 0 && !wait_all(&bar.k_full[nslot], phase_of(g + 1, 0))) { ok = false; break; }
+                tc_fence_after();
+                issue_qk_half(s, nslot, h, h == 0 ? &bar.s_ready[s] : &bar.s_b_ready[s],
+                              h == 1 && s == 1 && j + 2 == n);
+              }
+            }
+          }
+        }
+      } else {
       for (int j = 0; ok && j < n; ++j) {
         const int g = gstep + j;
         const bool more = j + 1 < n;
@@ -1123,6 +1419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_qk(s, nslot, s == 1 && j + 2 == n);
           }
         }
+      }
       }
       gstep += n;
       ++qcnt;
@@ -1172,7 +1469,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cls = tile_class<DECODE, BM>(a, w, s, t);
         if (!wait_spin_all(&bar.s_ready[s], (gstep + j) & 1)) { ok = false; break; }
         tc_fence_after();
-        softmax_step<D, DECODE, MOD, BM>(a, w, s, row, t, cls, tS, tO, j == 0, st, &bar.p_ready[s]);
+        if constexpr (!kHalfTiles<DECODE, MOD>) {
+          softmax_step<D, DECODE, MOD, BM>(a, w, s, row, t, cls, tS, tO, j == 0, st, &bar.p_ready[s]);
+        } else if (!softmax_step_halves<D, MOD, BM>(a, w, s, row, t, cls, tS, tO, j == 0, st, bar, gstep + j,
+                                                      abort_flag)) {
+          ok = false;
+          break;
+        }
         if (DECODE)
           tw.t += 2;
         else
