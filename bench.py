@@ -346,6 +346,66 @@ def _row_pairs(w: W.Prefill, i: int, d) -> int:
     return int(i - np.searchsorted(doc, doc[i]) + 1)
 
 
+# ---------------------------------------------------------------- ranks
+
+class RankGroup:
+    """The ranks of one run. Each rank processes its own batch (weak scaling,
+    no data-path collective); the group is used only for the barriers around
+    the timed region and for the max of the per-rank times. NCCL on GPUs;
+    the same calls work over gloo on CPU."""
+
+    def __init__(self, world: int = 1, rank: int = 0, local: int = 0, dist=None, device=None):
+        self.world, self.rank, self.local = world, rank, local
+        self.dist, self.device = dist, device
+
+    def barrier(self):
+        if self.dist is None:
+            return
+        if self.device is not None and self.device.type == "cuda":
+            self.dist.barrier(device_ids=[self.local])
+        else:
+            self.dist.barrier()
+
+    def max(self, x: float) -> float:
+        if self.dist is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.barrier()
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def init_ranks(backend: str, device=None, timeout_s: int = 120) -> RankGroup:
+    """Joins the process group described by RANK / LOCAL_RANK / WORLD_SIZE /
+    MASTER_ADDR / MASTER_PORT (torchrun's variables); world size 1 needs none."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world == 1:
+        return RankGroup(1, 0, local, None, device)
+    import datetime
+    import torch.distributed as dist
+    kw = {"device_id": device} if backend == "nccl" else {}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+    return RankGroup(world, rank, local, dist, device)
+
+
+def rank_seed_shift(rank: int) -> int:
+    """Each rank draws its own batch of the workload (same shapes, other seeds)."""
+    return 1000 * rank
+
+
+def weak_scaling_value(work_per_rank: float, world: int, t_max: float) -> float:
+    """Whole-job throughput: the work all ranks processed over the slowest rank's time."""
+    return work_per_rank * world / t_max
+
+
 # ---------------------------------------------------------------- main
 
 def reference_arm(args):
@@ -402,27 +462,12 @@ def main():
     import torch
     import exact_attention_145_b200 as ea
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier(device_ids=[local])
-
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = init_ranks("nccl", device)
+    world, rank = ranks.world, ranks.rank
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     peaks, peak_src = load_peaks()
     ea.load_library()
@@ -430,7 +475,7 @@ def main():
     w = W.WORKLOADS[args.workload]
 
     # ------------------------------------------------------------ primary: prefill
-    setup = prefill_setup(torch, ea, w, device, seed_shift=1000 * rank)
+    setup = prefill_setup(torch, ea, w, device, seed_shift=rank_seed_shift(rank))
     sampler = ClockSampler(physical_gpu_index(local)) if rank == 0 else None
     if sampler:
         sampler.start()
@@ -438,7 +483,7 @@ def main():
     if sampler:
         sampler.stop()
     t_max = max_over_ranks(t)
-    value = setup["flops"] * args.steps * world / t_max / 1e12
+    value = weak_scaling_value(setup["flops"] * args.steps, world, t_max) / 1e12
     launch_s = t / args.steps
     achieved = setup["flops"] / launch_s / 1e12
     peak = float(peaks["bf16_tflops"])
@@ -461,7 +506,7 @@ def main():
                        "parallelism": "independent replicas per GPU (no data-path collective)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "attn_fwd_kernel<128,false>",
+                         "kernel": "attn_fwd_kernel<128, prefill, no score mod, no block mask>",
                          "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % peak_src
                          if peak_src == "measured" else "fallback 1.59 PF/s"},
             "e2e": {"value": e2e_total, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -478,9 +523,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_prefill(w)
 
-    if dist is not None:
-        barrier()
-        dist.destroy_process_group()
+    ranks.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -491,11 +534,11 @@ def secondary(torch, ea, device, stream, peaks, rank, barrier, max_over_ranks, w
     launches = 0
     for name in ("window1024_softcap30_s8192", "packed_docs_alibi_s16384"):
         w = W.WORKLOADS[name]
-        s = prefill_setup(torch, ea, w, device, seed_shift=1000 * rank)
+        s = prefill_setup(torch, ea, w, device, seed_shift=rank_seed_shift(rank))
         t, _ = graph_time(torch, s["step"], steps, stream, 5, barrier)
         t = max_over_ranks(t)
         ach = s["flops"] / (t / steps) / 1e12
-        out[name] = {"value": ach * world, "unit": "TFLOP/s", "ms_per_step": 1e3 * t / steps, "pairs": s["pairs"],
+        out[name] = {"value": weak_scaling_value(s["flops"] * steps, world, t) / 1e12, "unit": "TFLOP/s", "ms_per_step": 1e3 * t / steps, "pairs": s["pairs"],
                      "roofline_frac": ach / float(peaks["bf16_tflops"])}
         launches += steps
         if s["bm"] is not None:
@@ -515,7 +558,7 @@ def secondary(torch, ea, device, stream, peaks, rank, barrier, max_over_ranks, w
             out[name]["block_mask_build_us"] = 1e6 * tb / 50
             launches += 50
     w = W.WORKLOADS["mqa_paged_decode_b32_kv32768"]
-    s = decode_setup(torch, ea, w, device, seed_shift=1000 * rank)
+    s = decode_setup(torch, ea, w, device, seed_shift=rank_seed_shift(rank))
     t, _ = graph_time(torch, s["step"], steps, stream, 5, barrier)
     t = max_over_ranks(t)
     gbs = s["bytes"] / (t / steps) / 1e9
