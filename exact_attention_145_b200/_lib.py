@@ -16,7 +16,7 @@ MOD_NONE, MOD_SOFTCAP, MOD_ALIBI = range(3)
 
 EXPORTS = ("attn_block_mask_bytes", "attn_block_mask_layout", "attn_build_block_mask", "attn_fwd",
            "attn_decode_num_splits", "attn_decode_workspace_bytes", "attn_decode", "attn_lse_combine",
-           "attn_status_str", "attn_decode_noalloc")
+           "attn_status_str", "attn_decode_noalloc", "attn_selftest_wait_timeout")
 ATTN_DECODE_NOALLOC_MAX_BYTES = 32 * 1024 * 1024
 
 c_i64x3 = ctypes.c_int64 * 3
@@ -94,6 +94,8 @@ def load() -> ctypes.CDLL:
         lib.attn_lse_combine.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_lse_combine.restype = ctypes.c_int
+        lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        lib.attn_selftest_wait_timeout.restype = ctypes.c_int
         lib.attn_status_str.argtypes = [ctypes.c_int]
         lib.attn_status_str.restype = ctypes.c_char_p
         _lib = lib

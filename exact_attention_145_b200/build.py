@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libattn.so")
-SOURCES = [os.path.join(CSRC, "attn_api.cu"), os.path.join(CSRC, "decode_noalloc.cu")]
+SOURCES = [os.path.join(CSRC, "attn_api.cu"), os.path.join(CSRC, "decode_noalloc.cu"), os.path.join(CSRC, "selftest.cu")]
 DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("fwd_kernel.cuh", "aux_kernels.cuh", "sm100.cuh")] + [
     os.path.join(ROOT, "include", "attn.h")]
 

@@ -197,6 +197,17 @@ attn_status attn_lse_combine(const float *o_parts, const float *lse_parts, int r
 #define ATTN_DECODE_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
 attn_status attn_decode_noalloc(const attn_decode_params *p, void *stream);
 
+/* Failure-detection self-test (no counterpart on the pages). Launches one
+ * warp that waits, with the bounded wait every pipeline barrier of these
+ * kernels uses, on a barrier nothing arrives on. After the wait's limit
+ * (about one second of SM clock) the kernel ORs ATTN_DEV_TIMEOUT into
+ * *status and exits normally; the context stays usable.
+ *  - status: device int (caller-owned), read by the caller after the stream
+ *    is synchronised.
+ *  - Returns ATTN_ERR_INVALID_ARG for a NULL status, ATTN_ERR_CUDA if the
+ *    launch fails, ATTN_OK otherwise. Asynchronous on the given stream. */
+attn_status attn_selftest_wait_timeout(int *status, void *stream);
+
 const char *attn_status_str(attn_status s);
 
 #ifdef __cplusplus

@@ -39,6 +39,10 @@ def test_library_exports_every_declared_symbol(lib):
         assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
 
 
+def test_selftest_rejects_a_null_status(lib):
+    assert lib.attn_selftest_wait_timeout(None, None) == _lib.ATTN_ERR_INVALID_ARG
+
+
 def test_status_strings(lib):
     assert lib.attn_status_str(0) == b"ok"
     assert lib.attn_status_str(4) == b"workspace too small"
