@@ -593,13 +593,24 @@ def profile_arm(args):
     return 0
 
 
-def kernel_source_sha() -> str:
+def code_digest(text: str) -> str:
+    """sha256 (16 hex digits) of C++ source with comments and whitespace removed,
+    so that editing a comment does not count as changing the kernel."""
     import hashlib
-    h = hashlib.sha256()
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = re.sub(r"\s+", "", text)
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
+
+
+def kernel_source_sha() -> str:
+    """Digest of the prefill kernel's code (fwd_kernel.cuh + sm100.cuh)."""
+    parts = []
     for f in ("exact_attention_145_b200/csrc/fwd_kernel.cuh", "exact_attention_145_b200/csrc/sm100.cuh"):
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
-    return h.hexdigest()[:16]
+        with open(os.path.join(ROOT, f)) as fh:
+            parts.append(fh.read())
+    return code_digest("\n".join(parts))
 
 
 def _traffic_from_profiles(workload: str):

@@ -17,20 +17,26 @@
 // softmax overlaps the other's MMAs: on B200 the exponentials take about
 // twice as long as the two GEMMs of a tile, so a single query tile per CTA
 // would leave the tensor cores idle ("FlexAttention + FlashAttention-4" talk,
-// the two-Q-tile ping-pong pipeline). MMA order per step:
+// the two-Q-tile ping-pong pipeline). MMA order per step, whole tiles
+// (decode, and prefill without a score mod):
 //   PV(0, j) QK(0, j+1) PV(1, j) QK(1, j+1)
-// TMEM (512 columns): S0 | S1 | O0 | O1. P (bf16) overwrites the first half of
-// its S region once the softmax has read S into registers, and feeds the PV
-// MMA straight from TMEM. tcgen05.mma ops of one thread execute in issue
-// order, so QK(s, j+1) overwrites S(s) only after PV(s, j) has read P(s).
+// Prefill with a score mod hands tiles over in key halves a (keys 0-63) and
+// b (keys 64-127), see "prefill, half tiles" below:
+//   PVa(0) QKa(0) PVa(1) QKa(1) PVb(0) QKb(0) PVb(1) QKb(1)
+// TMEM (512 columns): S0 | S1 | O0 | O1. P (bf16) overwrites part of its S
+// region once the softmax has read those scores into registers (columns
+// [0, 64) for whole tiles; [0, 32) and [64, 96) for half tiles) and feeds the
+// PV MMA straight from TMEM. tcgen05.mma ops of one thread execute in issue
+// order, so a QK^T overwrites S(s) only after the PV that reads P from it.
 //
 // Online softmax ("A Deep Dive into Flash Attention", section "2. Online
 // Softmax"), in base 2: x = log2(e) * score; each row keeps a reference max
 // m and a running sum l; O is rescaled by 2^(m_old - m_new) only when some
 // row of the warp sees its max grow by more than 8 (probabilities stay below
 // 2^8, which bf16 P and the fp32 accumulators absorb exactly as well).
-// Because QK(s, j+1) is committed after PV(s, j), seeing S(s, j+1) ready
-// implies O(s) is settled, so the rescale needs no extra wait.
+// With whole tiles QK(s, j+1) is committed after PV(s, j), so seeing
+// S(s, j+1) ready implies O(s) is settled and the rescale needs no extra
+// wait; half tiles wait for the one PV that may still be in flight.
 //
 // Prefill pairs the subtiles either as two query heads of one KV group over
 // the same 128 rows (GQA, group size even: identical masks, K/V shared) or as

@@ -1,0 +1,39 @@
+"""Host-side logic that needs no GPU: the decode split heuristic exported by
+the library and the bench's kernel-code digest (which decides whether the
+recorded DRAM traffic still describes the kernel)."""
+import pytest
+
+from exact_attention_145_b200 import _lib
+from exact_attention_145_b200.build import build
+
+import bench
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return _lib.load()
+
+
+def test_decode_splits_fill_one_wave_when_they_can(lib):
+    # 32 sequences x 1 KV head: 4 splits give 128 units, one wave of 148 SMs
+    assert lib.attn_decode_num_splits(32, 128, 1, 32768, 0) == 4
+    # a few long sequences: as many splits as fit one wave
+    assert lib.attn_decode_num_splits(4, 128, 1, 32768, 0) == 37
+    # sequences already fill the GPU: no split
+    assert lib.attn_decode_num_splits(148, 128, 1, 2048, 0) == 1
+    assert lib.attn_decode_num_splits(64, 64, 8, 4096, 0) == 1
+
+
+def test_decode_explicit_splits_are_clamped_to_key_tiles(lib):
+    assert lib.attn_decode_num_splits(2, 8, 1, 1000, 5) == 5
+    assert lib.attn_decode_num_splits(2, 8, 1, 1000, 64) == 8  # 1000 keys = 8 tiles of 128
+    assert lib.attn_decode_num_splits(0, 8, 1, 1000, 0) == 1
+
+
+def test_code_digest_ignores_comments_and_whitespace_only():
+    a = "int f(int x) {\n  return x + 1;  // one more\n}\n"
+    b = "/* header */ int f(int x) { return x + 1; }"
+    c = "int f(int x) { return x + 2; }"
+    assert bench.code_digest(a) == bench.code_digest(b)
+    assert bench.code_digest(a) != bench.code_digest(c)
