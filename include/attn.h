@@ -152,7 +152,11 @@ typedef struct {
   int *status;                /* optional device int, ATTN_DEV_* bits */
 } attn_decode_params;
 
-/* Number of splits attn_decode uses for these sizes (resolves num_splits = 0). */
+/* Number of splits attn_decode uses for these sizes (resolves num_splits = 0).
+ * An explicit num_splits is clamped to the number of 128-key tiles of
+ * max_seqlen. Automatic: the count minimising waves of CTAs x (tiles per split
+ * + a fixed per-unit cost of ten tiles), fewer splits on ties, so one full
+ * wave of (sequence, KV head, split) units is preferred when it fits. */
 int attn_decode_num_splits(int B, int Hq, int Hkv, int max_seqlen, int num_splits);
 
 /* Workspace bytes attn_decode needs: one fp32 partial O row and LSE per

@@ -37,3 +37,27 @@ def test_code_digest_ignores_comments_and_whitespace_only():
     c = "int f(int x) { return x + 2; }"
     assert bench.code_digest(a) == bench.code_digest(b)
     assert bench.code_digest(a) != bench.code_digest(c)
+
+
+@pytest.mark.parametrize("name", ["tiny_mha_s128_d64", "causal_gqa_llama8b_s2048", "window1024_softcap30_s8192",
+                                  "packed_docs_alibi_s16384"])
+def test_bench_flop_accounting_matches_the_oracle_pair_count(name):
+    """bench.py's closed-form pair counts (the FLOP numerator of every
+    TFLOP/s figure) against the oracle's brute-force count, on the workloads'
+    own masks at a reduced length where the workload allows it."""
+    import oracle
+    import workloads as W
+    w = W.WORKLOADS[name]
+    S = min(w.S, 3000)
+    ws = W.Prefill(**{**w.__dict__, "S": S})
+    doc_lens = None
+    kw = {}
+    if w.mask == W.MASK_CAUSAL:
+        kw = dict(window=(-1, 0))
+    elif w.mask == W.MASK_WINDOW:
+        kw = dict(window=(w.window_left, w.window_right))
+    elif w.mask == W.MASK_DOCUMENT:
+        doc_lens = W.doc_lengths(w.seed + 0x100, S, *w.doc_range)
+        kw = dict(doc_id=W.doc_ids_from_lengths(doc_lens))
+    per_head = oracle.count_pairs(w.mask, S, S, **kw)
+    assert bench.unmasked_pairs(ws, doc_lens) == per_head * w.B * w.Hq
