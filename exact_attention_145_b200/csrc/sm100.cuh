@@ -1,7 +1,8 @@
 // sm100.cuh - thin inline-PTX wrappers for the Blackwell (sm_100a) features the
-// attention kernels use: mbarriers with bounded waits, TMA tiled loads (never
-// with cluster multicast), tcgen05 tensor-memory allocation, load/store and
-// MMA issue, and the shared-memory matrix descriptors the MMAs read.
+// attention kernels use: mbarriers with bounded waits, TMA tiled loads (each
+// into the issuing CTA's own shared memory) and stores, tcgen05 tensor-memory
+// allocation, load/store and MMA issue, and the shared-memory matrix
+// descriptors the MMAs read.
 //
 // Every wait in this file is bounded: after kWaitTimeoutCycles SM cycles a
 // wait gives up, raises the CTA-wide abort flag and returns false, so that a
@@ -118,7 +119,8 @@ __device__ __forceinline__ bool mbar_wait_timeout(uint64_t* bar, uint32_t parity
 
 // ---------------------------------------------------------------- TMA
 // Tiled bulk-tensor loads, global -> this CTA's shared memory, completion
-// counted in bytes on an mbarrier. No multicast form exists in this file.
+// counted in bytes on an mbarrier. Every load here fills only the issuing
+// CTA's shared memory from this GPU's global memory.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
