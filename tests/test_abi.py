@@ -102,6 +102,13 @@ def test_fwd_bad_strides_and_document_mask(lib):
     p = _fwd_params()
     p.q_stride = _lib.c_i64x3(128 * 4 * 128, 4 * 128, 100)
     assert lib.attn_fwd(ctypes.byref(p), None) == _lib.ATTN_ERR_UNSUPPORTED
+    # a zero stride is refused on a dimension longer than 1 (rows would alias) ...
+    p = _fwd_params()
+    p.o_stride = _lib.c_i64x3(128 * 4 * 128, 4 * 128, 0)  # 4 heads, head stride 0
+    assert lib.attn_fwd(ctypes.byref(p), None) == _lib.ATTN_ERR_UNSUPPORTED
+    p = _fwd_params()
+    p.k_stride = _lib.c_i64x3(128 * 2 * 128, 0, 128)  # 128 keys, sequence stride 0
+    assert lib.attn_fwd(ctypes.byref(p), None) == _lib.ATTN_ERR_UNSUPPORTED
     p = _fwd_params()
     p.mask.kind = _lib.MASK_DOCUMENT  # no doc ids, no block mask
     assert lib.attn_fwd(ctypes.byref(p), None) == _lib.ATTN_ERR_INVALID_ARG
