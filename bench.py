@@ -300,10 +300,12 @@ def e2e_prefill(torch, ea, w: W.Prefill, setup, device, steps: int):
     return setup["flops"] * steps / t / 1e12, h2d, d2h
 
 
-def cpu_baseline_prefill(w: W.Prefill, seconds: float = 12.0):
-    """The oracle, as it stands, on a bounded sample of query rows of the workload."""
+def cpu_baseline_prefill(w: W.Prefill, seconds: float = 12.0, d=None, first_rows: int = 64):
+    """The oracle, as it stands, on a bounded sample of query rows of the
+    workload (inputs d generated once by the caller when given)."""
     import oracle
-    d = W.make_prefill_inputs(w)
+    if d is None:
+        d = W.make_prefill_inputs(w)
     kw = {}
     if w.mask == W.MASK_CAUSAL:
         kw = dict(mask=W.MASK_CAUSAL, window=(-1, 0))
@@ -317,7 +319,7 @@ def cpu_baseline_prefill(w: W.Prefill, seconds: float = 12.0):
         kw.update(mod=W.MOD_ALIBI, alibi=d["alibi"])
     threads = oracle.default_threads()
     rng = np.random.default_rng(0)
-    n = 64
+    n = first_rows
     total_flops, total_t, total_rows = 0, 0.0, 0
     while total_t < seconds:
         rows = np.stack([rng.integers(0, w.B, n), rng.integers(0, w.Hq, n), rng.integers(0, w.S, n)],
@@ -416,23 +418,32 @@ def reference_arm(args):
     import oracle
     w = W.WORKLOADS[PRIMARY]
     oracle.build()
+    d = W.make_prefill_inputs(w)
+    # Each step is a bounded sample of query rows, sized so that the whole
+    # run (warm-up included) takes about two minutes whatever K and W are.
+    per_step = min(2.0, max(0.002, 120.0 / max(args.steps + args.warmup, 1)))
+    rows = 64 if per_step >= 0.05 else 8
     for _ in range(args.warmup):
-        cpu_baseline_prefill(w, seconds=0.5)
+        cpu_baseline_prefill(w, seconds=per_step, d=d, first_rows=rows)
     t_steps = []
     vals = []
+    total_rows = 0
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        cb = cpu_baseline_prefill(w, seconds=max(0.5, 20.0 / max(args.steps, 1)))
+        cb = cpu_baseline_prefill(w, seconds=per_step, d=d, first_rows=rows)
         t_steps.append(time.perf_counter() - t0)
         vals.append(cb["value"])
+        total_rows += int(cb["sample"].split()[0])
     value = float(np.mean(vals))
+    sample = ("%d steps, each a bounded sample of random query rows of %s (about %.3f s of fp64 C oracle time "
+              "on %d threads); %d rows in total" % (args.steps, w.name, per_step, cb["cores"], total_rows))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(t_steps)),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": PRIMARY, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "D": w.D,
                        "mask": "causal", "step": "bounded sample of query rows"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cb["cores"], "kind": "oracle",
-                             "sample": cb["sample"]},
+                             "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
