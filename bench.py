@@ -408,6 +408,65 @@ def weak_scaling_value(work_per_rank: float, world: int, t_max: float) -> float:
     return work_per_rank * world / t_max
 
 
+def _free_port() -> int:
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def launch_plan(gpus: int, env) -> str:
+    """How this process runs `--gpus N`: "single" (N == 1, no process group),
+    "rank" (already one of torchrun's N ranks), or "spawn" (N > 1 and no
+    torchrun around us: relaunch this command under torch.distributed.run).
+    A WORLD_SIZE that disagrees with --gpus is an error."""
+    world = env.get("WORLD_SIZE")
+    if world is None:
+        return "spawn" if gpus > 1 else "single"
+    if int(world) != gpus:
+        raise SystemExit("bench.py: --gpus %d but WORLD_SIZE=%s; run N ranks with --gpus N" % (gpus, world))
+    return "rank" if gpus > 1 else "single"
+
+
+def spawn_ranks(gpus: int, argv, timeout_s: int = 1800) -> int:
+    """Re-runs this script as `gpus` ranks of one node (torch.distributed.run,
+    rendezvous on 127.0.0.1) and returns the launcher's exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=%d" % gpus,
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), os.path.abspath(__file__)] + list(argv)
+    try:
+        return subprocess.run(cmd, timeout=timeout_s).returncode
+    except subprocess.TimeoutExpired:
+        sys.stderr.write("bench.py: ranks did not finish within %d s\n" % timeout_s)
+        return 124
+
+
+def plumbing_check(args) -> int:
+    """CPU rehearsal of a multi-rank run (gloo): every rank draws its own
+    batch of the workload, the barrier and the max over ranks run as in the
+    GPU path, and rank 0 prints one JSON line with the world size, each rank's
+    input digest and the slowest rank's (synthetic) time."""
+    import hashlib
+    group = init_ranks("gloo", timeout_s=120)
+    w = W.WORKLOADS[args.workload]
+    mine = W.Prefill(**{**w.__dict__, "seed": w.seed + rank_seed_shift(group.rank)})
+    q = W.make_prefill_inputs(mine, S=128)["q"]
+    digest = hashlib.sha256(q.tobytes()).hexdigest()[:16]
+    group.barrier()
+    t_max = group.max(1.0 + 0.25 * group.rank)
+    digests = [digest]
+    if group.dist is not None:
+        digests = [None] * group.world
+        group.dist.all_gather_object(digests, digest)
+    world = group.world
+    group.close()
+    if group.rank == 0:
+        print(json.dumps({"plumbing": True, "n_gpus": world, "gpus_flag": args.gpus, "rank_input_digests": digests,
+                          "t_max": t_max, "value": weak_scaling_value(1.0, world, t_max)}), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------- main
 
 def reference_arm(args):
@@ -462,13 +521,21 @@ def main():
     ap.add_argument("--secondary-steps", type=int, default=200)
     ap.add_argument("--profile", default=None, choices=list(W.WORKLOADS) + ["block_mask"],
                     help="run --steps eager steps of one workload (for ncu captures); prints no JSON line")
+    ap.add_argument("--plumbing-check", action="store_true",
+                    help="CPU only: rehearse the N-rank launch, barrier and max over ranks over gloo")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus < 1:
+        raise SystemExit("bench.py: --gpus must be at least 1")
     if args.impl == "reference":
         return reference_arm(args)
     if args.profile:
         return profile_arm(args)
+    if launch_plan(args.gpus, os.environ) == "spawn":
+        return spawn_ranks(args.gpus, sys.argv[1:])
+    if args.plumbing_check:
+        return plumbing_check(args)
 
     import torch
     import exact_attention_145_b200 as ea

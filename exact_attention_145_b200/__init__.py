@@ -20,12 +20,12 @@ import ctypes
 from typing import Optional, Tuple
 
 from . import _lib
-from ._lib import (ATTN_DEV_BAD_PAGE, ATTN_DEV_TIMEOUT, MASK_CAUSAL, MASK_DOCUMENT, MASK_NONE, MASK_WINDOW,
+from ._lib import (ATTN_DEV_BAD_LEN, ATTN_DEV_BAD_PAGE, ATTN_DEV_TIMEOUT, MASK_CAUSAL, MASK_DOCUMENT, MASK_NONE, MASK_WINDOW,
                    MOD_ALIBI, MOD_NONE, MOD_SOFTCAP, AttnError)
 
 __all__ = ["attn_fwd", "attn_decode", "attn_decode_noalloc", "attn_build_block_mask", "attn_lse_combine",
            "BlockMask", "AttnError",
-           "load_library", "ATTN_DEV_TIMEOUT", "ATTN_DEV_BAD_PAGE"]
+           "load_library", "ATTN_DEV_TIMEOUT", "ATTN_DEV_BAD_PAGE", "ATTN_DEV_BAD_LEN"]
 
 
 def load_library():
@@ -194,39 +194,33 @@ def attn_fwd(q, k, v, *, scale: Optional[float] = None, causal: bool = False, wi
     return out, lse
 
 
-def attn_decode(q, k_cache, v_cache, block_table, cache_seqlens, *, max_seqlen: Optional[int] = None,
-                scale: Optional[float] = None, softcap: Optional[float] = None, alibi_slopes=None,
-                num_splits: int = 0, out=None, lse=None, workspace=None, status=None, with_lse: bool = True,
-                stream=None):
-    """Split-KV decode over a paged cache. q [B, Hq, D] (or [B, 1, Hq, D]);
-    k_cache/v_cache [num_pages, page_size, Hkv, D]; block_table int32
-    [B, max_pages]; cache_seqlens int32 [B]. Returns (O [B, Hq, D], LSE [B, Hq])."""
+def _decode_params(q, k_cache, v_cache, block_table, cache_seqlens, max_seqlen, scale, softcap, alibi_slopes,
+                   num_splits, out, lse, status):
+    """Checks the decode inputs and fills the C parameter block (shared by
+    attn_decode and attn_decode_noalloc)."""
     torch = _torch()
     if q.dim() == 4:
         q = q[:, 0]
     _check_bf16("q", q, 3)
     _check_bf16("k_cache", k_cache, 4)
     _check_bf16("v_cache", v_cache, 4)
-    if k_cache.stride() != v_cache.stride():
-        raise ValueError("k_cache and v_cache must share strides")
+    if k_cache.shape != v_cache.shape or k_cache.stride() != v_cache.stride():
+        raise ValueError("k_cache and v_cache must share shape and strides")
     for name, t in (("block_table", block_table), ("cache_seqlens", cache_seqlens)):
         if t.dtype != torch.int32 or not t.is_cuda:
             raise ValueError("%s must be an int32 CUDA tensor" % name)
-    if block_table.stride(1) != 1 or not cache_seqlens.is_contiguous():
+    if block_table.dim() != 2 or block_table.stride(1) != 1 or not cache_seqlens.is_contiguous():
         raise ValueError("block_table rows and cache_seqlens must be contiguous")
     B, Hq, D = q.shape
-    P, page, Hkv, _ = k_cache.shape
+    P, page, Hkv, Dk = k_cache.shape
+    if Dk != D or block_table.shape[0] != B or cache_seqlens.numel() != B:
+        raise ValueError("q, caches, block_table and cache_seqlens disagree on B or D")
+    if out is not None and (tuple(out.shape) != (B, Hq, D) or out.dtype != torch.bfloat16):
+        raise ValueError("out must be bf16 [B, Hq, D]")
+    if lse is not None and (tuple(lse.shape) != (B, Hq) or lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise ValueError("lse must be contiguous fp32 [B, Hq]")
     if max_seqlen is None:
         max_seqlen = block_table.shape[1] * page
-    lib = _lib.load()
-    splits = lib.attn_decode_num_splits(B, Hq, Hkv, int(max_seqlen), int(num_splits))
-    need = lib.attn_decode_workspace_bytes(B, Hq, D, splits)
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    if out is None:
-        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
-    if lse is None and with_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     p = _lib.DecodeParams()
     p.q = q.data_ptr()
     p.q_stride = _lib.c_i64x2(q.stride(0), q.stride(1))
@@ -239,10 +233,33 @@ def attn_decode(q, k_cache, v_cache, block_table, cache_seqlens, *, max_seqlen: 
     p.scale = 0.0 if scale is None else float(scale)
     p.mod, p.softcap, p.alibi_slopes, p.alibi_batch_stride = _mod_args(softcap, alibi_slopes, Hq)
     p.num_splits = int(num_splits)
-    p.o = out.data_ptr()
-    p.o_stride = _lib.c_i64x2(out.stride(0), out.stride(1))
     p.lse = _ptr(lse)
     p.status = _ptr(status)
+    return p, q
+
+
+def attn_decode(q, k_cache, v_cache, block_table, cache_seqlens, *, max_seqlen: Optional[int] = None,
+                scale: Optional[float] = None, softcap: Optional[float] = None, alibi_slopes=None,
+                num_splits: int = 0, out=None, lse=None, workspace=None, status=None, with_lse: bool = True,
+                stream=None):
+    """Split-KV decode over a paged cache. q [B, Hq, D] (or [B, 1, Hq, D]);
+    k_cache/v_cache [num_pages, page_size, Hkv, D]; block_table int32
+    [B, max_pages]; cache_seqlens int32 [B]. Returns (O [B, Hq, D], LSE [B, Hq])."""
+    torch = _torch()
+    B, Hq, D = (q.shape[0], q.shape[-2], q.shape[-1])
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and with_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    p, q = _decode_params(q, k_cache, v_cache, block_table, cache_seqlens, max_seqlen, scale, softcap,
+                          alibi_slopes, num_splits, out, lse, status)
+    lib = _lib.load()
+    splits = lib.attn_decode_num_splits(p.B, p.Hq, p.Hkv, p.max_seqlen, p.num_splits)
+    need = lib.attn_decode_workspace_bytes(p.B, p.Hq, p.D, splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    p.o = out.data_ptr()
+    p.o_stride = _lib.c_i64x2(out.stride(0), out.stride(1))
     h = _stream_handle(q.device) if stream is None else stream
     _lib.check(lib.attn_decode(ctypes.byref(p), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                h), "attn_decode")
@@ -250,30 +267,17 @@ def attn_decode(q, k_cache, v_cache, block_table, cache_seqlens, *, max_seqlen: 
 
 
 def attn_decode_noalloc(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, *, max_seqlen: int,
-                        scale: Optional[float] = None, num_splits: int = 0, status=None, stream=None):
+                        scale: Optional[float] = None, softcap: Optional[float] = None, alibi_slopes=None,
+                        num_splits: int = 0, status=None, stream=None):
     """attn_decode whose split partials live in a fixed 32 MiB array inside the
     library, for callers that may not allocate device memory (out and lse are
     the caller's). Calls that would need more scratch raise AttnError
     (workspace too small). The first call on a device should precede any
     stream capture; calls that overlap on the GPU share the array and race."""
-    if q.dim() == 4:
-        q = q[:, 0]
-    p = _lib.DecodeParams()
-    p.q = q.data_ptr()
-    p.q_stride = _lib.c_i64x2(q.stride(0), q.stride(1))
-    p.k_cache, p.v_cache = k_cache.data_ptr(), v_cache.data_ptr()
-    p.cache_stride = _lib.c_i64x3(*k_cache.stride()[:3])
-    p.block_table, p.block_table_stride = block_table.data_ptr(), block_table.stride(0)
-    p.cache_seqlens = cache_seqlens.data_ptr()
-    p.B, p.Hq, p.D = q.shape
-    p.num_pages, p.page_size, p.Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
-    p.max_seqlen = int(max_seqlen)
-    p.scale = 0.0 if scale is None else float(scale)
-    p.num_splits = int(num_splits)
+    p, q = _decode_params(q, k_cache, v_cache, block_table, cache_seqlens, max_seqlen, scale, softcap,
+                          alibi_slopes, num_splits, out, lse, status)
     p.o = out.data_ptr()
     p.o_stride = _lib.c_i64x2(out.stride(0), out.stride(1))
-    p.lse = _ptr(lse)
-    p.status = _ptr(status)
     h = _stream_handle(q.device) if stream is None else stream
     _lib.check(_lib.load().attn_decode_noalloc(ctypes.byref(p), h), "attn_decode_noalloc")
     return out, lse

@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libattn.so")
 
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_WORKSPACE = range(5)
-ATTN_DEV_TIMEOUT, ATTN_DEV_BAD_PAGE = 1, 2
+ATTN_DEV_TIMEOUT, ATTN_DEV_BAD_PAGE, ATTN_DEV_BAD_LEN = 1, 2, 4
 MASK_NONE, MASK_CAUSAL, MASK_WINDOW, MASK_DOCUMENT = range(4)
 MOD_NONE, MOD_SOFTCAP, MOD_ALIBI = range(3)
 

@@ -445,6 +445,7 @@ attn_status attn_decode(const attn_decode_params* p, void* workspace, size_t wor
   const int tiles = (p->max_seqlen + kKeys - 1) / kKeys;
   a.n_splits = splits;
   a.tiles_per_split = (tiles + splits - 1) / splits;
+  a.max_seqlen = p->max_seqlen;
   const size_t rows = (size_t)p->B * p->Hq * splits;
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((rows * p->D * 4 + 255) & ~size_t(255)));

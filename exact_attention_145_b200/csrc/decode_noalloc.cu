@@ -20,7 +20,10 @@
 //  - The first call on each device does a one-time set-up: it looks up the
 //    device address of the array (cudaGetSymbolAddress), which may also load
 //    the library's device code on that device. Make that first call before
-//    any stream capture on the device.
+//    any stream capture on the device. The address is remembered together
+//    with the CUDA context it belongs to; if that context is replaced (after
+//    cudaDeviceReset, say), the next call repeats the set-up in the new one,
+//    and so should come before any capture as well.
 //  - Every call on a device uses the same array, which keeps whatever the
 //    previous call left there. Nothing in it has to start at zero: every
 //    partial the combine step reads is written by the same call first. Calls
@@ -28,6 +31,7 @@
 //    threads without ordering) race on the array and corrupt each other's
 //    results; issue them in order on one stream.
 //  - Nothing here allocates or frees device memory.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -41,21 +45,58 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
-void* g_scratch_addr[kMaxDevices] = {};  // device address of g_decode_scratch, per device
+// Per device: the device address of g_decode_scratch and the context in
+// which it was looked up.
+struct ScratchSlot {
+  CUcontext ctx;
+  void* addr;
+};
+ScratchSlot g_slots[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// cuCtxGetCurrent through the runtime's driver entry-point lookup, so the
+// library needs no link-time dependency on libcuda.
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<CtxGetCurrentFn>(nullptr);
+    return reinterpret_cast<CtxGetCurrentFn>(f);
+  }();
+  return fn;
+}
 
 // Host code cannot use g_decode_scratch directly: on the host that name is
-// only a stand-in for the device variable, so its device address is looked
-// up once per device, with that device current, and cached.
+// only a stand-in for the device variable. Its device address is looked up
+// with the device current and cached with the current context; a different
+// context (the old one was reset) triggers a fresh lookup, so a stale
+// address is never handed to a kernel.
 attn_status scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  CtxGetCurrentFn get = ctx_get_current();
+  if (!get) return ATTN_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return ATTN_ERR_CUDA;
+  if (ctx == nullptr) {
+    // No context is current yet: the symbol lookup initialises the device's
+    // primary context (it allocates nothing), after which it is current.
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_decode_scratch) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (get(&ctx) != CUDA_SUCCESS || ctx == nullptr) return ATTN_ERR_CUDA;
+  }
+  ScratchSlot& slot = g_slots[dev];
+  if (slot.addr == nullptr || slot.ctx != ctx) {
     void* addr = nullptr;
     if (cudaGetSymbolAddress(&addr, g_decode_scratch) != cudaSuccess || addr == nullptr) return ATTN_ERR_CUDA;
-    g_scratch_addr[dev] = addr;
+    slot.ctx = ctx;
+    slot.addr = addr;
   }
-  *out = g_scratch_addr[dev];
+  *out = slot.addr;
   return ATTN_OK;
 }
 

@@ -70,7 +70,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 enum : int { MASK_NONE = 0, MASK_CAUSAL = 1, MASK_WINDOW = 2, MASK_DOCUMENT = 3 };
 enum : int { MOD_NONE = 0, MOD_SOFTCAP = 1, MOD_ALIBI = 2 };
-enum : int { DEV_TIMEOUT = 1, DEV_BAD_PAGE = 2 };
+enum : int { DEV_TIMEOUT = 1, DEV_BAD_PAGE = 2, DEV_BAD_LEN = 4 };
 
 struct FwdArgs {
   int B, Hq, Hkv, Sq, Skv, g;
@@ -97,6 +97,7 @@ struct FwdArgs {
   int bt_stride;
   const int32_t* seqlens;
   int page_size, num_pages, box_rows, n_splits, tiles_per_split;
+  int max_seqlen;   // upper bound on cache_seqlens[b]; larger lengths are clamped and reported
   float* part_o;    // [B][Hq][n_splits][D]
   float* part_lse;  // [B][Hq][n_splits]
   int* status;
@@ -166,8 +167,10 @@ __device__ __forceinline__ Work map_work(const FwdArgs& a, int u) {
     w.b = bh / a.Hkv;
     w.head0 = w.head1 = w.hk * a.g;
     w.row00 = w.row01 = 0;
-    w.seqlen = a.seqlens[w.b];
-    const int nt = (max(w.seqlen, 0) + kKeys - 1) / kKeys;
+    // Keys past max_seqlen would fall outside the splits (and possibly the
+    // block table); such lengths are clamped here and reported by the producer.
+    w.seqlen = min(max(a.seqlens[w.b], 0), a.max_seqlen);
+    const int nt = (w.seqlen + kKeys - 1) / kKeys;
     w.t_begin = min(nt, w.split * a.tiles_per_split);
     w.t_end = min(nt, w.t_begin + a.tiles_per_split);
   } else {
@@ -536,16 +539,26 @@ __device__ __forceinline__ bool mask_chunk(const FwdArgs& a, const MaskRow& m, i
   if (BM && a.mask == MASK_DOCUMENT) {
     const int kv = t * kKeys + 32 * c;
     const int4* d4 = reinterpret_cast<const int4*>(a.doc_id + kv);
-    const int n4 = max(min(32, a.Skv - kv), 0) / 4;
+    // keys of this chunk inside the sequence: whole groups of four are read
+    // as one 16-byte load, a ragged last group (Skv not a multiple of 4)
+    // element by element; keys past Skv fail the span test below anyway.
+    const int nval = max(min(32, a.Skv - kv), 0);
+    const int n4 = nval / 4, tail = nval % 4;
 #pragma unroll
     for (int i4 = 0; i4 < 8; ++i4) {
       // volatile: keeps the load inside its chunk instead of letting all 32
       // of a tile be hoisted (and spilled) ahead of the loop
       int4 d = make_int4(-1, -1, -1, -1);
-      if (i4 < n4)
+      if (i4 < n4) {
         asm volatile("ld.global.nc.v4.s32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(d.x), "=r"(d.y), "=r"(d.z), "=r"(d.w)
                      : "l"(d4 + i4));
+      } else if (i4 == n4 && tail > 0) {
+        const int32_t* dp = a.doc_id + kv + 4 * i4;
+        d.x = __ldg(dp);
+        if (tail > 1) d.y = __ldg(dp + 1);
+        if (tail > 2) d.z = __ldg(dp + 2);
+      }
       const int j = 32 * c + 4 * i4;
       x[4 * i4 + 0] = (!m.none && (unsigned)(j + 0 - m.clo) <= m.span && d.x == m.dq) ? x[4 * i4 + 0] : NEG_INF;
       x[4 * i4 + 1] = (!m.none && (unsigned)(j + 1 - m.clo) <= m.span && d.y == m.dq) ? x[4 * i4 + 1] : NEG_INF;
@@ -1220,6 +1233,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = unit_of(r);
       if (u < 0) continue;
       const Work w = map_work<DECODE>(a, u);
+      if constexpr (DECODE) {
+        // one report per sequence: a length outside [0, max_seqlen]
+        const int raw = a.seqlens[w.b];
+        if (w.split == 0 && w.hk == 0 && (raw < 0 || raw > a.max_seqlen) && a.status && elect_one_sync())
+          atomicOr(a.status, DEV_BAD_LEN);
+        __syncwarp();
+      }
       TileWalker tw;
       const int n = walker_init<DECODE, BM>(a, w, tw);
       if (n == 0) continue;

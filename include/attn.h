@@ -49,6 +49,9 @@ typedef enum {
 /* Bits the kernels OR into *status. */
 #define ATTN_DEV_TIMEOUT 1   /* a bounded pipeline wait gave up; outputs invalid */
 #define ATTN_DEV_BAD_PAGE 2  /* a block_table entry was outside [0, num_pages) */
+#define ATTN_DEV_BAD_LEN 4   /* decode: a cache_seqlens[b] was negative or above max_seqlen;
+                                that sequence was computed over its first max_seqlen keys
+                                (none if negative) and its outputs are not the requested ones */
 
 /* Mask kinds (FlexAttention mask_mod equivalents, attention-gym issue 101 and
  * the FA4 talk; flash_attn window_size in the FlashAttention overview).
@@ -139,7 +142,9 @@ typedef struct {
   int block_table_stride;     /* >= max pages any sequence uses */
   const int32_t *cache_seqlens; /* int32 [B]: keys of sequence b are its first cache_seqlens[b] tokens */
   int B, Hq, Hkv, D, page_size, num_pages;
-  int max_seqlen;             /* upper bound on every cache_seqlens[b] (sizes the split) */
+  int max_seqlen;             /* upper bound on every cache_seqlens[b] (sizes the splits); a
+                                 larger or negative length is clamped to [0, max_seqlen] and
+                                 reported as ATTN_DEV_BAD_LEN in *status */
   float scale;                /* <= 0 selects 1/sqrt(D) */
   attn_mod_kind mod;          /* the query sits at position cache_seqlens[b] - 1 */
   float softcap;

@@ -120,6 +120,17 @@ def test_documents_alibi_gqa():
     full_case(1, S, 3, 3, 64, seed=81, doc_id_np=doc)
 
 
+@pytest.mark.parametrize("S", [129, 130, 131, 387])
+def test_documents_ragged_tail(S):
+    """Sequence lengths that are not a multiple of 4: the last group of
+    document ids is partial. Documents start inside the last key tile, so the
+    final rows depend on those ids."""
+    lens = [S - 3, 1, 2] if S < 200 else [100, 150, S - 250 - 1, 1]
+    doc = W.doc_ids_from_lengths(lens)
+    full_case(1, S, 4, 2, 128, seed=85 + S, doc_id_np=doc)
+    full_case(1, S, 2, 2, 64, seed=86 + S, doc_id_np=doc, alibi_np=W.alibi_slopes(2))
+
+
 def test_bhsd_strided_inputs():
     B, S, H, D = 2, 260, 4, 128
     q = W.normal_bf16(90, (B, H, S, D))
@@ -266,6 +277,48 @@ def test_decode_mods_and_d64():
                                    mod=W.MOD_ALIBI, alibi=sl)
     o, lse, st = run_decode(d, 8, alibi_np=sl)
     compare(o, o_ref, lse, lse_ref, "decode alibi")
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(128, 1), (8, 2)])
+@pytest.mark.parametrize("mod", ["alibi", "softcap"])
+def test_decode_mods_grouped_heads(Hq, Hkv, mod):
+    """Score mods when several query heads share a KV head: in decode each MMA
+    row is a different query head (row r of KV head hk is head hk*g + r), so the
+    ALiBi slope must follow the row. MQA (g = 128) and GQA (g = 4)."""
+    w = W.Decode("t", B=3, Hq=Hq, Hkv=Hkv, D=128, kv_len=1500, page_size=128, seed=135 + Hq + Hkv)
+    d = W.make_decode_inputs(w, seqlens=np.array([1500, 700, 129], np.int32))
+    if mod == "alibi":
+        sl = W.alibi_slopes(Hq)
+        okw, kw = dict(mod=W.MOD_ALIBI, alibi=sl), dict(alibi_np=sl)
+    else:
+        okw, kw = dict(mod=W.MOD_SOFTCAP, softcap=5.0), dict(softcap=5.0)
+    o_ref, lse_ref = oracle.decode(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["cache_seqlens"], **okw)
+    o, lse, st = run_decode(d, Hkv, **kw)
+    assert st == 0
+    compare(o, o_ref, lse, lse_ref, "decode %s g=%d" % (mod, Hq // Hkv))
+
+
+def test_decode_length_above_max_seqlen_is_reported_and_clamped():
+    """A cache_seqlens entry above max_seqlen (or negative) sets ATTN_DEV_BAD_LEN;
+    the other sequences stay exact and the bad one is computed over its first
+    max_seqlen keys. Made on the host: nothing faults."""
+    w = W.Decode("t", B=3, Hq=8, Hkv=1, D=128, kv_len=1024, page_size=128, seed=145)
+    d = W.make_decode_inputs(w, seqlens=np.array([1024, 600, 300], np.int32))
+    o, lse, st = run_decode(d, 1, max_seqlen=600)
+    assert st & ea.ATTN_DEV_BAD_LEN and not st & ea.ATTN_DEV_BAD_PAGE
+    clamped = d["cache_seqlens"].copy()
+    clamped[0] = 600
+    o_ref, lse_ref = oracle.decode(d["q"], d["k_cache"], d["v_cache"], d["block_table"], clamped)
+    compare(o, o_ref, lse, lse_ref, "decode clamped")
+    d2 = dict(d, cache_seqlens=np.array([-5, 600, 300], np.int32))
+    o, lse, st = run_decode(d2, 1, max_seqlen=600)
+    assert st & ea.ATTN_DEV_BAD_LEN
+    assert np.all(o[0] == 0) and np.all(lse[0] == -np.inf)
+    o_ref, lse_ref = oracle.decode(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["cache_seqlens"])
+    compare(o[1:], o_ref[1:], lse[1:], lse_ref[1:], "decode negative length")
+    # within bounds: no report
+    _, _, st = run_decode(d, 1, max_seqlen=1024)
+    assert st == 0
 
 
 def test_decode_zero_length_sequence():

@@ -82,3 +82,32 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
 
     assert bench.reference_arm(Args) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_launch_plan_follows_gpus_and_world_size():
+    import bench
+    assert bench.launch_plan(1, {}) == "single"
+    assert bench.launch_plan(2, {}) == "spawn"
+    assert bench.launch_plan(4, {"WORLD_SIZE": "4"}) == "rank"
+    assert bench.launch_plan(1, {"WORLD_SIZE": "1"}) == "single"
+    with pytest.raises(SystemExit):
+        bench.launch_plan(8, {"WORLD_SIZE": "2"})
+
+
+def test_bench_gpus_two_launches_two_ranks_with_their_own_batches():
+    """`bench.py --gpus 2` without torchrun relaunches itself as two ranks;
+    the CPU rehearsal (gloo) shows world 2, two different input batches and
+    the slowest rank's time."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_PORT")}
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--plumbing-check"],
+                         capture_output=True, text=True, timeout=300, env=env, cwd=root)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [json.loads(x) for x in res.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    line = lines[0]
+    assert line["n_gpus"] == 2 and line["gpus_flag"] == 2
+    assert len(line["rank_input_digests"]) == 2 and len(set(line["rank_input_digests"])) == 2
+    assert line["t_max"] == 1.25 and abs(line["value"] - 2 / 1.25) < 1e-12

@@ -224,6 +224,54 @@ def test_alibi_zero_slope_is_plain_and_per_batch_slopes():
     assert np.array_equal(o3[1], o1[1]) and not np.allclose(o3[0, :, :3], o1[0, :, :3])
 
 
+def _geometric_lse(slope, n):
+    """ln sum_{d=0}^{n-1} exp(-slope * d): the log-sum-exp of a causal row whose
+    raw scores are all 0, so that only the ALiBi bias slope * (kv - q) remains."""
+    if slope == 0.0:
+        return math.log(n)
+    return math.log(-math.expm1(-slope * n)) - math.log(-math.expm1(-slope))
+
+
+def test_alibi_slope_is_indexed_by_query_head():
+    # FlashAttention overview, "Examples": alibi_slopes has shape (nheads,) with
+    # nheads the number of query heads, so under GQA each query head uses its
+    # own slope, not the one of the KV head it shares. Raw scores are 0 (q = 0),
+    # Hq = 4 query heads share one KV head, and every row's LSE has the
+    # geometric closed form of its own head's slope. An oracle that indexed the
+    # slope by the KV head would give all four heads the first slope.
+    S, Hq, D = 40, 4, 8
+    q = np.zeros((1, S, Hq, D), np.uint16)
+    k = W.normal_bf16(141, (1, S, 1, D))
+    v = W.normal_bf16(142, (1, S, 1, D))
+    slopes = np.array([0.5, 0.125, 0.03125, 0.0], np.float32)
+    o, lse = oracle.attn(q, k, v, mask=W.MASK_CAUSAL, window=(-1, 0), mod=W.MOD_ALIBI, alibi=slopes)
+    for h in range(Hq):
+        for i in (0, 1, 7, S - 1):
+            assert abs(lse[0, h, i] - _geometric_lse(float(slopes[h]), i + 1)) < 1e-13, (h, i)
+    # only head 0 has a non-zero slope: heads 1..3 must equal the plain result
+    o_plain, l_plain = oracle.attn(q, k, v, mask=W.MASK_CAUSAL, window=(-1, 0))
+    one = np.array([0.5, 0.0, 0.0, 0.0], np.float32)
+    o1, l1 = oracle.attn(q, k, v, mask=W.MASK_CAUSAL, window=(-1, 0), mod=W.MOD_ALIBI, alibi=one)
+    assert np.array_equal(o1[:, :, 1:], o_plain[:, :, 1:]) and np.array_equal(l1[:, 1:], l_plain[:, 1:])
+    assert not np.allclose(o1[:, 1:, 0], o_plain[:, 1:, 0])
+
+
+def test_decode_alibi_slope_is_indexed_by_query_head():
+    # The same reading for the paged decode: the single query of sequence b sits
+    # at position cache_seqlens[b] - 1 and head h adds slope[h] * (t - (n - 1)).
+    Hq, D, page = 4, 8, 16
+    seqlens = np.array([37, 5], np.int32)
+    w = W.Decode("t", B=2, Hq=Hq, Hkv=1, D=D, kv_len=48, page_size=page, seed=143)
+    d = W.make_decode_inputs(w, seqlens=seqlens)
+    q0 = np.zeros_like(d["q"])
+    slopes = np.array([0.5, 0.125, 0.03125, 0.0], np.float32)
+    _, lse = oracle.decode(q0, d["k_cache"], d["v_cache"], d["block_table"], d["cache_seqlens"],
+                           mod=W.MOD_ALIBI, alibi=slopes)
+    for b, n in enumerate(seqlens):
+        for h in range(Hq):
+            assert abs(lse[b, h] - _geometric_lse(float(slopes[h]), int(n))) < 1e-13, (b, h)
+
+
 def test_alibi_slopes_for_eight_heads():
     assert np.array_equal(W.alibi_slopes(8), np.array(golden()["alibi8"], np.float32))
     s32 = W.alibi_slopes(32)
