@@ -20,12 +20,14 @@ import ctypes
 from typing import Optional, Tuple
 
 from . import _lib
-from ._lib import (ATTN_DEV_BAD_LEN, ATTN_DEV_BAD_PAGE, ATTN_DEV_TIMEOUT, MASK_CAUSAL, MASK_DOCUMENT, MASK_NONE, MASK_WINDOW,
+from ._lib import (ATTN_DEV_BAD_LEN, ATTN_DEV_BAD_MASK, ATTN_DEV_BAD_PAGE, ATTN_DEV_TIMEOUT, MASK_CAUSAL,
+                   MASK_DOCUMENT, MASK_NONE, MASK_WINDOW,
                    MOD_ALIBI, MOD_NONE, MOD_SOFTCAP, AttnError)
 
 __all__ = ["attn_fwd", "attn_decode", "attn_decode_noalloc", "attn_build_block_mask", "attn_lse_combine",
            "BlockMask", "AttnError",
-           "load_library", "ATTN_DEV_TIMEOUT", "ATTN_DEV_BAD_PAGE", "ATTN_DEV_BAD_LEN"]
+           "load_library", "ATTN_DEV_TIMEOUT", "ATTN_DEV_BAD_PAGE", "ATTN_DEV_BAD_LEN",
+           "ATTN_DEV_BAD_MASK"]
 
 
 def load_library():
@@ -61,23 +63,24 @@ def _check_bf16(name, t, ndim):
 class BlockMask:
     """Tile-level mask (FlexAttention BlockMask equivalent) in one device buffer.
 
-    cls[q_tile, kv_tile] is 0 (empty), 1 (partial) or 2 (full); part_idx /
-    full_idx list the partial / full kv tiles of each q tile in ascending order,
-    the first part_cnt / full_cnt entries of each row being valid.
+    cls[b, h, q_tile, kv_tile] is 0 (empty), 1 (partial) or 2 (full); part_idx /
+    full_idx list the partial / full kv tiles of each (b, h, q tile) in
+    ascending order, the first part_cnt / full_cnt entries of each row being
+    valid. Bm / Hm of 1 mean one slice shared by every batch / head.
     """
 
-    def __init__(self, Sq: int, Skv: int, blk_q: int, blk_kv: int, device):
+    def __init__(self, Sq: int, Skv: int, blk_q: int, blk_kv: int, device, Bm: int = 1, Hm: int = 1):
         torch = _torch()
         lib = _lib.load()
-        nbytes = lib.attn_block_mask_bytes(Sq, Skv, blk_q, blk_kv)
+        nbytes = lib.attn_block_mask_bytes(Bm, Hm, Sq, Skv, blk_q, blk_kv)
         if nbytes == 0:
             raise ValueError("invalid block mask sizes")
         self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.c = _lib.BlockMaskC()
-        _lib.check(lib.attn_block_mask_layout(self.buffer.data_ptr(), nbytes, Sq, Skv, blk_q, blk_kv,
+        _lib.check(lib.attn_block_mask_layout(self.buffer.data_ptr(), nbytes, Bm, Hm, Sq, Skv, blk_q, blk_kv,
                                               ctypes.byref(self.c)), "attn_block_mask_layout")
-        self.Sq, self.Skv, self.blk_q, self.blk_kv = Sq, Skv, blk_q, blk_kv
-        self.shape = (self.c.n_q_tiles, self.c.n_kv_tiles)
+        self.Bm, self.Hm, self.Sq, self.Skv, self.blk_q, self.blk_kv = Bm, Hm, Sq, Skv, blk_q, blk_kv
+        self.shape = (Bm, Hm, self.c.n_q_tiles, self.c.n_kv_tiles)
 
     def _view(self, addr, dtype, shape):
         torch = _torch()
@@ -94,11 +97,11 @@ class BlockMask:
 
     @property
     def part_cnt(self):
-        return self._view(self.c.part_cnt, _torch().int32, (self.shape[0],))
+        return self._view(self.c.part_cnt, _torch().int32, self.shape[:3])
 
     @property
     def full_cnt(self):
-        return self._view(self.c.full_cnt, _torch().int32, (self.shape[0],))
+        return self._view(self.c.full_cnt, _torch().int32, self.shape[:3])
 
     @property
     def part_idx(self):
@@ -107,6 +110,31 @@ class BlockMask:
     @property
     def full_idx(self):
         return self._view(self.c.full_idx, _torch().int32, self.shape)
+
+    @property
+    def row_order(self):
+        """[Bm, n_q_tiles]: q-tiles by decreasing visited kv tiles (work order)."""
+        return self._view(self.c.row_order, _torch().int32, (self.Bm, self.shape[2]))
+
+    @property
+    def doc_start(self):
+        """[Bm, Sq]: first position of each position's run of equal document ids."""
+        return self._view(self.c.doc_start, _torch().int32, (self.Bm, self.Sq))
+
+    @property
+    def doc_sorted(self):
+        """[Bm]: 1 where the document ids never decrease."""
+        return self._view(self.c.doc_sorted, _torch().int32, (self.Bm,))
+
+
+def _doc_rows(doc_id):
+    """(pointer, batch stride in elements) of a doc_id tensor [S] or [B, S]."""
+    torch = _torch()
+    if doc_id is None:
+        return None, 0
+    if doc_id.dtype != torch.int32 or not doc_id.is_cuda or doc_id.stride(-1) != 1 or doc_id.dim() not in (1, 2):
+        raise ValueError("doc_id must be an int32 CUDA tensor [S] or [B, S] with contiguous rows")
+    return doc_id.data_ptr(), (doc_id.stride(0) if doc_id.dim() == 2 else 0)
 
 
 def _mask_spec(causal: bool, window, q_offset: int, doc_id) -> Tuple[_lib.MaskSpec, int]:
@@ -121,20 +149,29 @@ def _mask_spec(causal: bool, window, q_offset: int, doc_id) -> Tuple[_lib.MaskSp
     else:
         kind = MASK_NONE
     spec.kind, spec.window_left, spec.window_right, spec.q_offset = kind, wl, wr, int(q_offset)
-    spec.doc_id = _ptr(doc_id)
+    spec.doc_id, spec.doc_batch_stride = _doc_rows(doc_id)
     return spec, kind
 
 
 def attn_build_block_mask(Sq: int, Skv: int, *, causal: bool = False, window=None, q_offset: int = 0,
-                          doc_id=None, blk_q: int = 128, blk_kv: int = 128, device=None, stream=None) -> BlockMask:
-    """Classify every (q-tile, kv-tile) of the mask on the device."""
+                          doc_id=None, B: Optional[int] = None, H: int = 1, blk_q: int = 128, blk_kv: int = 128,
+                          device=None, stream=None) -> BlockMask:
+    """Classify every (batch, head, q-tile, kv-tile) of the mask on the device
+    (FlexAttention create_block_mask(mask_mod, B, H, Q_LEN, KV_LEN, BLOCK_SIZE)).
+    doc_id [S] gives one slice shared by every batch, [B, S] one slice per
+    batch; B defaults to the rows of doc_id (1 otherwise) and H to 1 (shared by
+    every head)."""
     torch = _torch()
     if doc_id is not None:
-        if doc_id.dtype != torch.int32 or not doc_id.is_cuda or not doc_id.is_contiguous():
-            raise ValueError("doc_id must be a contiguous int32 CUDA tensor")
+        _doc_rows(doc_id)
         device = doc_id.device
+        if B is None:
+            B = doc_id.shape[0] if doc_id.dim() == 2 else 1
+        if doc_id.dim() == 2 and doc_id.shape[0] != B:
+            raise ValueError("doc_id has %d rows but B = %d" % (doc_id.shape[0], B))
+    B = 1 if B is None else int(B)
     device = device if device is not None else torch.device("cuda")
-    bm = BlockMask(Sq, Skv, blk_q, blk_kv, device)
+    bm = BlockMask(Sq, Skv, blk_q, blk_kv, device, Bm=B, Hm=int(H))
     spec, _ = _mask_spec(causal, window, q_offset, doc_id)
     h = _stream_handle(device) if stream is None else stream
     _lib.check(_lib.load().attn_build_block_mask(ctypes.byref(spec), ctypes.byref(bm.c), h),

@@ -8,9 +8,20 @@ import threading
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libattn.so")
+TRACE_LIB_PATH = os.path.join(HERE, "libattn_trace.so")
+
+
+def lib_path() -> str:
+    """libattn.so, or with ATTN_LIBRARY_VARIANT=trace (set before the first
+    call) the cycle-trace build libattn_trace.so: the same kernels plus trace
+    records at the pipeline hand-offs (see trace.py). ATTN_LIBRARY=<path>
+    loads another build of the same C ABI instead."""
+    if os.environ.get("ATTN_LIBRARY"):
+        return os.path.abspath(os.environ["ATTN_LIBRARY"])
+    return TRACE_LIB_PATH if os.environ.get("ATTN_LIBRARY_VARIANT") == "trace" else LIB_PATH
 
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_WORKSPACE = range(5)
-ATTN_DEV_TIMEOUT, ATTN_DEV_BAD_PAGE, ATTN_DEV_BAD_LEN = 1, 2, 4
+ATTN_DEV_TIMEOUT, ATTN_DEV_BAD_PAGE, ATTN_DEV_BAD_LEN, ATTN_DEV_BAD_MASK = 1, 2, 4, 8
 MASK_NONE, MASK_CAUSAL, MASK_WINDOW, MASK_DOCUMENT = range(4)
 MOD_NONE, MOD_SOFTCAP, MOD_ALIBI = range(3)
 
@@ -25,14 +36,16 @@ c_i64x2 = ctypes.c_int64 * 2
 
 class MaskSpec(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("window_left", ctypes.c_int), ("window_right", ctypes.c_int),
-                ("q_offset", ctypes.c_int), ("doc_id", ctypes.c_void_p)]
+                ("q_offset", ctypes.c_int), ("doc_id", ctypes.c_void_p), ("doc_batch_stride", ctypes.c_int64)]
 
 
 class BlockMaskC(ctypes.Structure):
-    _fields_ = [("Sq", ctypes.c_int), ("Skv", ctypes.c_int), ("blk_q", ctypes.c_int), ("blk_kv", ctypes.c_int),
+    _fields_ = [("Bm", ctypes.c_int), ("Hm", ctypes.c_int),
+                ("Sq", ctypes.c_int), ("Skv", ctypes.c_int), ("blk_q", ctypes.c_int), ("blk_kv", ctypes.c_int),
                 ("n_q_tiles", ctypes.c_int), ("n_kv_tiles", ctypes.c_int),
                 ("cls", ctypes.c_void_p), ("part_cnt", ctypes.c_void_p), ("part_idx", ctypes.c_void_p),
-                ("full_cnt", ctypes.c_void_p), ("full_idx", ctypes.c_void_p)]
+                ("full_cnt", ctypes.c_void_p), ("full_idx", ctypes.c_void_p),
+                ("row_order", ctypes.c_void_p), ("doc_start", ctypes.c_void_p), ("doc_sorted", ctypes.c_void_p)]
 
 
 class FwdParams(ctypes.Structure):
@@ -70,13 +83,15 @@ def load() -> ctypes.CDLL:
     with _lock:
         if _lib is not None:
             return _lib
-        if not os.path.exists(LIB_PATH):
+        path = lib_path()
+        if not os.path.exists(path):
             raise RuntimeError(
-                "libattn.so is not built (expected at %s); run `python -m exact_attention_145_b200.build`" % LIB_PATH)
-        lib = ctypes.CDLL(LIB_PATH)
-        lib.attn_block_mask_bytes.argtypes = [ctypes.c_int] * 4
+                "%s is not built (expected at %s); run `python -m exact_attention_145_b200.build`"
+                % (os.path.basename(path), path))
+        lib = ctypes.CDLL(path)
+        lib.attn_block_mask_bytes.argtypes = [ctypes.c_int] * 6
         lib.attn_block_mask_bytes.restype = ctypes.c_size_t
-        lib.attn_block_mask_layout.argtypes = [ctypes.c_void_p, ctypes.c_size_t] + [ctypes.c_int] * 4 + [
+        lib.attn_block_mask_layout.argtypes = [ctypes.c_void_p, ctypes.c_size_t] + [ctypes.c_int] * 6 + [
             ctypes.POINTER(BlockMaskC)]
         lib.attn_block_mask_layout.restype = ctypes.c_int
         lib.attn_build_block_mask.argtypes = [ctypes.POINTER(MaskSpec), ctypes.POINTER(BlockMaskC), ctypes.c_void_p]
@@ -96,6 +111,9 @@ def load() -> ctypes.CDLL:
         lib.attn_lse_combine.restype = ctypes.c_int
         lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_selftest_wait_timeout.restype = ctypes.c_int
+        if hasattr(lib, "attn_trace_configure"):
+            lib.attn_trace_configure.argtypes = [ctypes.c_void_p, ctypes.c_int]
+            lib.attn_trace_configure.restype = ctypes.c_int
         lib.attn_status_str.argtypes = [ctypes.c_int]
         lib.attn_status_str.restype = ctypes.c_char_p
         _lib = lib

@@ -22,26 +22,32 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+# The cycle-trace variant (-DATTN_TRACE): the same kernels with trace records
+# at the pipeline hand-offs, plus attn_trace_configure. Used by trace.py only.
+TRACE_LIB = os.path.join(HERE, "libattn_trace.so")
+
+
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in DEPENDS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if force or stale():
-        tmp = LIB + ".tmp.%d" % os.getpid()
-        cmd = [nvcc()] + NVCC_FLAGS + ["-o", tmp] + SOURCES
+def build(force: bool = False, verbose: bool = False, trace: bool = False) -> str:
+    lib = TRACE_LIB if trace else LIB
+    if force or stale(lib):
+        tmp = lib + ".tmp.%d" % os.getpid()
+        cmd = [nvcc()] + NVCC_FLAGS + (["-DATTN_TRACE"] if trace else []) + ["-o", tmp] + SOURCES
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             sys.stderr.write(res.stdout + res.stderr)
-            raise RuntimeError("nvcc failed building libattn.so")
+            raise RuntimeError("nvcc failed building %s" % os.path.basename(lib))
         if verbose:
             sys.stderr.write(res.stderr)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, trace="--trace" in sys.argv))

@@ -34,6 +34,23 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+#ifdef ATTN_TRACE
+// Trace buffer of the ATTN_TRACE build (attn_trace_configure); every launch
+// of the forward kernel records into it.
+uint2* g_trace = nullptr;
+int g_trace_per_role = 0;
+#endif
+
+void set_trace(FwdArgs& a) {
+#ifdef ATTN_TRACE
+  a.trace = g_trace;
+  a.trace_per_role = g_trace_per_role;
+#else
+  a.trace = nullptr;
+  a.trace_per_role = 0;
+#endif
+}
+
 // A bf16 tensor map over (dims[0] contiguous, dims[1..r-1] with element
 // strides), box = {64, box_rows, 1, ...}, 128-byte swizzle.
 attn_status make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const int64_t* strides_el,
@@ -173,22 +190,27 @@ const char* attn_status_str(attn_status s) {
   return "unknown status";
 }
 
-size_t attn_block_mask_bytes(int Sq, int Skv, int blk_q, int blk_kv) {
-  if (Sq <= 0 || Skv <= 0 || blk_q <= 0 || blk_kv <= 0) return 0;
+size_t attn_block_mask_bytes(int Bm, int Hm, int Sq, int Skv, int blk_q, int blk_kv) {
+  if (Bm <= 0 || Hm <= 0 || Sq <= 0 || Skv <= 0 || blk_q <= 0 || blk_kv <= 0) return 0;
+  const size_t slices = (size_t)Bm * Hm;
   const size_t nQ = (Sq + blk_q - 1) / blk_q, nK = (Skv + blk_kv - 1) / blk_kv;
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  return up(nQ * nK) + 2 * up(nQ * 4) + 2 * up(nQ * nK * 4);
+  return up(slices * nQ * nK) + 2 * up(slices * nQ * 4) + 2 * up(slices * nQ * nK * 4) + up((size_t)Bm * nQ * 4) +
+         up((size_t)Bm * Sq * 4) + up((size_t)Bm * 4);
 }
 
-attn_status attn_block_mask_layout(void* buf, size_t buf_bytes, int Sq, int Skv, int blk_q, int blk_kv,
-                                   attn_block_mask* out) {
+attn_status attn_block_mask_layout(void* buf, size_t buf_bytes, int Bm, int Hm, int Sq, int Skv, int blk_q,
+                                   int blk_kv, attn_block_mask* out) {
   if (!out || !buf || !aligned16(buf)) return ATTN_ERR_INVALID_ARG;
-  const size_t need = attn_block_mask_bytes(Sq, Skv, blk_q, blk_kv);
+  const size_t need = attn_block_mask_bytes(Bm, Hm, Sq, Skv, blk_q, blk_kv);
   if (need == 0) return ATTN_ERR_INVALID_ARG;
   if (buf_bytes < need) return ATTN_ERR_WORKSPACE;
+  const size_t slices = (size_t)Bm * Hm;
   const size_t nQ = (Sq + blk_q - 1) / blk_q, nK = (Skv + blk_kv - 1) / blk_kv;
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   uint8_t* p = static_cast<uint8_t*>(buf);
+  out->Bm = Bm;
+  out->Hm = Hm;
   out->Sq = Sq;
   out->Skv = Skv;
   out->blk_q = blk_q;
@@ -196,34 +218,51 @@ attn_status attn_block_mask_layout(void* buf, size_t buf_bytes, int Sq, int Skv,
   out->n_q_tiles = static_cast<int>(nQ);
   out->n_kv_tiles = static_cast<int>(nK);
   out->cls = p;
-  p += up(nQ * nK);
+  p += up(slices * nQ * nK);
   out->part_cnt = reinterpret_cast<int32_t*>(p);
-  p += up(nQ * 4);
+  p += up(slices * nQ * 4);
   out->full_cnt = reinterpret_cast<int32_t*>(p);
-  p += up(nQ * 4);
+  p += up(slices * nQ * 4);
   out->part_idx = reinterpret_cast<int32_t*>(p);
-  p += up(nQ * nK * 4);
+  p += up(slices * nQ * nK * 4);
   out->full_idx = reinterpret_cast<int32_t*>(p);
+  p += up(slices * nQ * nK * 4);
+  out->row_order = reinterpret_cast<int32_t*>(p);
+  p += up((size_t)Bm * nQ * 4);
+  out->doc_start = reinterpret_cast<int32_t*>(p);
+  p += up((size_t)Bm * Sq * 4);
+  out->doc_sorted = reinterpret_cast<int32_t*>(p);
   return ATTN_OK;
 }
 
 attn_status attn_build_block_mask(const attn_mask_spec* spec, const attn_block_mask* out, void* stream) {
   if (!spec || !out) return ATTN_ERR_INVALID_ARG;
-  if (out->Sq <= 0 || out->Skv <= 0 || out->blk_q <= 0 || out->blk_kv <= 0) return ATTN_ERR_INVALID_ARG;
+  if (out->Bm <= 0 || out->Hm <= 0 || out->Sq <= 0 || out->Skv <= 0 || out->blk_q <= 0 || out->blk_kv <= 0)
+    return ATTN_ERR_INVALID_ARG;
   if (out->blk_q % 16 || out->blk_kv % 16 || out->blk_q > 1024 || out->blk_kv > 1024) return ATTN_ERR_UNSUPPORTED;
+  if (out->Bm > 65535 || (long)out->Bm * out->Hm * ((out->Sq + out->blk_q - 1) / out->blk_q) > 0x7fffffffL)
+    return ATTN_ERR_UNSUPPORTED;
   if (out->n_q_tiles != (out->Sq + out->blk_q - 1) / out->blk_q ||
       out->n_kv_tiles != (out->Skv + out->blk_kv - 1) / out->blk_kv)
     return ATTN_ERR_INVALID_ARG;
-  if (!out->cls || !out->part_cnt || !out->part_idx || !out->full_cnt || !out->full_idx) return ATTN_ERR_INVALID_ARG;
-  if (spec->kind < ATTN_MASK_NONE || spec->kind > ATTN_MASK_DOCUMENT) return ATTN_ERR_INVALID_ARG;
-  if (spec->kind == ATTN_MASK_DOCUMENT && (!spec->doc_id || out->Sq != out->Skv || spec->q_offset != 0))
+  if (!out->cls || !out->part_cnt || !out->part_idx || !out->full_cnt || !out->full_idx || !out->row_order)
     return ATTN_ERR_INVALID_ARG;
+  if (spec->kind == ATTN_MASK_DOCUMENT && (!out->doc_start || !out->doc_sorted)) return ATTN_ERR_INVALID_ARG;
+  if (spec->kind < ATTN_MASK_NONE || spec->kind > ATTN_MASK_DOCUMENT) return ATTN_ERR_INVALID_ARG;
+  if (spec->kind == ATTN_MASK_DOCUMENT) {
+    if (!spec->doc_id || out->Sq != out->Skv || spec->q_offset != 0) return ATTN_ERR_INVALID_ARG;
+    if (spec->doc_batch_stride < 0 || (spec->doc_batch_stride > 0 && spec->doc_batch_stride < out->Sq))
+      return ATTN_ERR_INVALID_ARG;
+  }
   MaskArgs a;
   a.kind = spec->kind;
   a.wl = spec->kind == ATTN_MASK_CAUSAL ? -1 : spec->window_left;
   a.wr = spec->kind == ATTN_MASK_CAUSAL ? 0 : spec->window_right;
   a.q_offset = spec->kind == ATTN_MASK_NONE ? 0 : spec->q_offset;
   a.doc_id = spec->doc_id;
+  a.doc_bstride = spec->kind == ATTN_MASK_DOCUMENT ? spec->doc_batch_stride : 0;
+  a.Bm = out->Bm;
+  a.Hm = out->Hm;
   a.Sq = out->Sq;
   a.Skv = out->Skv;
   a.blk_q = out->blk_q;
@@ -235,15 +274,25 @@ attn_status attn_build_block_mask(const attn_mask_spec* spec, const attn_block_m
   a.part_idx = out->part_idx;
   a.full_cnt = out->full_cnt;
   a.full_idx = out->full_idx;
+  a.row_order = out->row_order;
+  a.doc_start = out->doc_start;
+  a.doc_sorted = out->doc_sorted;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Pass 1 classifies head slice 0 of every batch slice (the mask kinds do not
+  // depend on the head); pass 2 copies it to the other head slices and builds
+  // every slice's lists. A mask that does not depend on the batch either
+  // (no per-batch document rows) is classified once and copied.
+  const int b_class = (a.kind == ATTN_MASK_DOCUMENT && a.doc_bstride > 0) ? a.Bm : 1;
   if (a.kind == ATTN_MASK_DOCUMENT) {
     const size_t smem = (size_t)kKvPerCta * a.blk_kv * sizeof(int);
-    classify_doc_kernel<<<dim3(a.nQ, (a.nK + kKvPerCta - 1) / kKvPerCta), kMaskThreads, smem, st>>>(a);
+    classify_doc_kernel<<<dim3(a.nQ, (a.nK + kKvPerCta - 1) / kKvPerCta, b_class), kMaskThreads, smem, st>>>(a);
   } else {
     const int64_t tiles = (int64_t)a.nQ * a.nK;
     classify_range_kernel<<<(unsigned)((tiles + 255) / 256), 256, 0, st>>>(a);
   }
-  compact_lists_kernel<<<a.nQ, 32, 0, st>>>(a);
+  compact_lists_kernel<<<dim3(a.nQ, a.Bm * a.Hm), 32, 0, st>>>(a, b_class);
+  row_order_kernel<<<a.Bm, kOrderThreads, 0, st>>>(a);
+  if (a.kind == ATTN_MASK_DOCUMENT) doc_runs_kernel<<<a.Bm, kRunThreads, 0, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -265,7 +314,10 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
   const int nK = (p->Skv + kKeys - 1) / kKeys;
   if (p->mask.kind == ATTN_MASK_DOCUMENT) {
     if (!p->mask.doc_id || p->Sq != p->Skv || p->mask.q_offset != 0 || !p->block_mask) return ATTN_ERR_INVALID_ARG;
-    if (!aligned16(p->mask.doc_id)) return ATTN_ERR_UNSUPPORTED;  // read as int4 by the kernel
+    if (p->mask.doc_batch_stride < 0 || (p->mask.doc_batch_stride > 0 && p->mask.doc_batch_stride < p->Sq))
+      return ATTN_ERR_INVALID_ARG;
+    // rows are read as int4 by the kernel
+    if (!aligned16(p->mask.doc_id) || p->mask.doc_batch_stride % 4) return ATTN_ERR_UNSUPPORTED;
   }
   if (p->block_mask) {
     const attn_block_mask* bm = p->block_mask;
@@ -273,6 +325,8 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
         bm->n_q_tiles != nQ || bm->n_kv_tiles != nK || !bm->part_cnt || !bm->part_idx || !bm->full_cnt ||
         !bm->full_idx)
       return ATTN_ERR_INVALID_ARG;
+    if ((bm->Bm != 1 && bm->Bm != p->B) || (bm->Hm != 1 && bm->Hm != p->Hq)) return ATTN_ERR_INVALID_ARG;
+    if (p->mask.kind == ATTN_MASK_DOCUMENT && (!bm->doc_start || !bm->doc_sorted)) return ATTN_ERR_INVALID_ARG;
   }
 
   FwdArgs a{};
@@ -306,8 +360,14 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
       a.q_offset = 0;
   }
   a.doc_id = p->mask.doc_id;
+  a.doc_bstride = p->mask.kind == ATTN_MASK_DOCUMENT ? p->mask.doc_batch_stride : 0;
   a.bm_cls = p->block_mask ? p->block_mask->cls : nullptr;
   if (p->block_mask) {
+    a.bm_Bm = p->block_mask->Bm;
+    a.bm_Hm = p->block_mask->Hm;
+    a.bm_row_order = p->block_mask->row_order;
+    a.bm_doc_start = p->block_mask->doc_start;
+    a.bm_doc_sorted = p->block_mask->doc_sorted;
     a.bm_part_cnt = p->block_mask->part_cnt;
     a.bm_part_idx = p->block_mask->part_idx;
     a.bm_full_cnt = p->block_mask->full_cnt;
@@ -343,6 +403,7 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
   // O is written in 32-row boxes, one per softmax warp.
   if (attn_status st = make_map(&mo, p->o, 4, dq, so, 32, 1)) return st;
 
+  set_trace(a);
   const int HU = a.pair_heads ? a.Hq / 2 : a.Hq;
   const long units = (long)a.B * HU * a.n_row_units;
   if (units <= 0 || units > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
@@ -460,6 +521,7 @@ attn_status attn_decode(const attn_decode_params* p, void* workspace, size_t wor
   if (attn_status st = make_map(&mk, p->k_cache, 4, dc, sc, (uint32_t)a.box_rows, 2)) return st;
   if (attn_status st = make_map(&mv, p->v_cache, 4, dc, sc, (uint32_t)a.box_rows, 2)) return st;
 
+  set_trace(a);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long units = (long)p->B * p->Hkv * splits;
   if (units > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
@@ -504,5 +566,17 @@ attn_status attn_lse_combine(const float* o_parts, const float* lse_parts, int r
   c.lse = lse;
   return launch_combine(c, D, static_cast<cudaStream_t>(stream));
 }
+
+#ifdef ATTN_TRACE
+// Trace builds only: every later forward launch appends cycle records to buf
+// (device memory, grid CTAs x 10 roles x per_role uint2 records; the caller
+// zeroes it). buf = NULL turns tracing off.
+attn_status attn_trace_configure(void* buf, int per_role) {
+  if (buf != nullptr && per_role <= 0) return ATTN_ERR_INVALID_ARG;
+  g_trace = static_cast<uint2*>(buf);
+  g_trace_per_role = buf ? per_role : 0;
+  return ATTN_OK;
+}
+#endif
 
 }  // extern "C"

@@ -11,9 +11,14 @@ namespace attn_kernels {
 struct MaskArgs {
   int kind, wl, wr, q_offset;
   const int32_t* doc_id;
+  int64_t doc_bstride;  // elements between the document rows of batches; 0 = one shared row
+  int Bm, Hm;           // batch and head slices of the tables: [Bm][Hm][nQ][nK]
   int Sq, Skv, blk_q, blk_kv, nQ, nK;
   uint8_t* cls;
   int32_t *part_cnt, *part_idx, *full_cnt, *full_idx;
+  int32_t* row_order;   // [Bm][nQ]
+  int32_t* doc_start;   // [Bm][Sq] (document masks)
+  int32_t* doc_sorted;  // [Bm]     (document masks)
 };
 
 // Block-mask build, pass 1: classify tiles (0 empty, 1 partial, 2 full).
@@ -66,10 +71,14 @@ __device__ __forceinline__ void warp_minmax(int& lo, int& hi) {
 // any tile when the ids are not grouped) are evaluated pair by pair: each
 // thread walks its query rows against the tile's keys, stopping once it has
 // seen both an allowed and a masked pair, and block votes give "any" and "all".
-__global__ void __launch_bounds__(kMaskThreads) classify_doc_kernel(const MaskArgs a) {
+// Batch slice b = blockIdx.z reads document row b and writes head slice 0 of
+// batch slice b.
+__global__ void __launch_bounds__(kMaskThreads) classify_doc_kernel(MaskArgs a) {
   extern __shared__ int doc_k[];  // [kKvPerCta * blk_kv] key doc ids
   __shared__ int red_lo[kMaskThreads / 32], red_hi[kMaskThreads / 32];
   __shared__ int tile_lo[kKvPerCta], tile_hi[kKvPerCta];
+  a.doc_id += (int64_t)blockIdx.z * a.doc_bstride;
+  a.cls += (int64_t)blockIdx.z * a.Hm * a.nQ * a.nK;
   const int qt = blockIdx.x;
   const int kt0 = blockIdx.y * kKvPerCta;
   const int kt1 = min(kt0 + kKvPerCta, a.nK);
@@ -152,28 +161,110 @@ __global__ void __launch_bounds__(kMaskThreads) classify_doc_kernel(const MaskAr
   }
 }
 
-// Pass 2: one warp per q-tile compacts the class row into the ascending
-// partial and full lists with ballots.
-__global__ void __launch_bounds__(32) compact_lists_kernel(const MaskArgs a) {
+// Pass 2: one warp per (slice, q-tile) compacts the class row into the
+// ascending partial and full lists with ballots. Pass 1 classified head slice
+// 0 of the first b_class batch slices; every other slice copies its class row
+// from head slice 0 of batch slice (b < b_class ? b : 0) first.
+__global__ void __launch_bounds__(32) compact_lists_kernel(const MaskArgs a, int b_class) {
   const int qt = blockIdx.x;
+  const int slice = blockIdx.y;  // b * Hm + h
+  const int b = slice / a.Hm;
   const int lane = threadIdx.x;
-  const uint8_t* row = a.cls + (int64_t)qt * a.nK;
+  const int64_t tiles = (int64_t)a.nQ * a.nK;
+  uint8_t* row = a.cls + slice * tiles + (int64_t)qt * a.nK;
+  const uint8_t* src = a.cls + (int64_t)(b < b_class ? b : 0) * a.Hm * tiles + (int64_t)qt * a.nK;
+  const bool copy = src != row;
+  int32_t* pidx = a.part_idx + slice * tiles + (int64_t)qt * a.nK;
+  int32_t* fidx = a.full_idx + slice * tiles + (int64_t)qt * a.nK;
   int np = 0, nf = 0;
   for (int k0 = 0; k0 < a.nK; k0 += 32) {
     const int kt = k0 + lane;
-    const uint8_t c = kt < a.nK ? row[kt] : 0;
+    const uint8_t c = kt < a.nK ? src[kt] : 0;
+    if (copy && kt < a.nK) row[kt] = c;
     const unsigned mp = __ballot_sync(0xffffffffu, c == 1);
     const unsigned mf = __ballot_sync(0xffffffffu, c == 2);
     const unsigned below = (1u << lane) - 1u;
-    if (c == 1) a.part_idx[(int64_t)qt * a.nK + np + __popc(mp & below)] = kt;
-    if (c == 2) a.full_idx[(int64_t)qt * a.nK + nf + __popc(mf & below)] = kt;
+    if (c == 1) pidx[np + __popc(mp & below)] = kt;
+    if (c == 2) fidx[nf + __popc(mf & below)] = kt;
     np += __popc(mp);
     nf += __popc(mf);
   }
   if (lane == 0) {
-    a.part_cnt[qt] = np;
-    a.full_cnt[qt] = nf;
+    a.part_cnt[(int64_t)slice * a.nQ + qt] = np;
+    a.full_cnt[(int64_t)slice * a.nQ + qt] = nf;
   }
+}
+
+// Pass 3: the work order of batch slice b = blockIdx.x: its q-tiles by
+// decreasing number of visited kv tiles (head slice 0), ties by index, so the
+// persistent attention kernel hands out the longest rows first. Each thread
+// ranks its q-tiles by counting the tiles that come before them.
+constexpr int kOrderThreads = 256;
+__global__ void __launch_bounds__(kOrderThreads) row_order_kernel(const MaskArgs a) {
+  const int b = blockIdx.x;
+  const int64_t base = (int64_t)b * a.Hm * a.nQ;  // head slice 0 of batch slice b
+  for (int i = threadIdx.x; i < a.nQ; i += blockDim.x) {
+    const int wi = a.part_cnt[base + i] + a.full_cnt[base + i];
+    int rank = 0;
+    for (int j = 0; j < a.nQ; ++j) {
+      const int wj = a.part_cnt[base + j] + a.full_cnt[base + j];
+      rank += (wj > wi) || (wj == wi && j < i);
+    }
+    a.row_order[(int64_t)b * a.nQ + rank] = i;
+  }
+}
+
+// Document masks, batch slice b = blockIdx.x (document row b, or row 0 when
+// the rows are shared): doc_start[i] = first position of the run of equal
+// ids that holds i, and doc_sorted = 1 when the ids never decrease (then
+// every document is a single run and key j <= i is allowed iff
+// j >= doc_start[i]). Each thread scans a contiguous chunk; the chunks'
+// last run starts are combined with a block-wide max scan.
+constexpr int kRunThreads = 1024;
+__global__ void __launch_bounds__(kRunThreads) doc_runs_kernel(const MaskArgs a) {
+  __shared__ int warp_max[kRunThreads / 32];
+  const int b = blockIdx.x;
+  const int32_t* doc = a.doc_id + (int64_t)b * a.doc_bstride;
+  int32_t* out = a.doc_start + (int64_t)b * a.Sq;
+  const int S = a.Sq;
+  const int chunk = (S + kRunThreads - 1) / kRunThreads;
+  const int i0 = min(S, (int)threadIdx.x * chunk), i1 = min(S, i0 + chunk);
+  int last = -1;
+  bool decreasing = false;
+  for (int i = i0; i < i1; ++i) {
+    const int d = doc[i];
+    if (i == 0 || d != doc[i - 1]) last = i;
+    if (i > 0 && d < doc[i - 1]) decreasing = true;
+  }
+  // inclusive max scan of `last` over threads: warps, then the warp totals
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  int incl = last;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl = max(incl, v);
+  }
+  if (lane == 31) warp_max[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_max[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w = max(w, v);
+    }
+    warp_max[lane] = w;  // inclusive over warps 0..lane
+  }
+  __syncthreads();
+  const int before_warp = warp > 0 ? warp_max[warp - 1] : -1;
+  const int excl_lane = __shfl_up_sync(0xffffffffu, incl, 1);
+  int cur = max(before_warp, lane > 0 ? excl_lane : -1);  // last run start before this chunk
+  for (int i = i0; i < i1; ++i) {
+    if (i == 0 || doc[i] != doc[i - 1]) cur = i;
+    out[i] = cur;
+  }
+  const int any_dec = __syncthreads_or(decreasing ? 1 : 0);
+  if (threadIdx.x == 0) a.doc_sorted[b] = any_dec ? 0 : 1;
 }
 
 // One warp per output row: lse = ln sum_i exp(lse_i); o = sum_i exp(lse_i - lse) o_i.

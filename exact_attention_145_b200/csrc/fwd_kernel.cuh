@@ -62,15 +62,17 @@ constexpr int kThreads = 384;
 constexpr int kSoftmaxRegs = 224;
 constexpr int kControlRegs = 56;  // warps 8-11, one warpgroup, one count
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split exceeds launch budget");
-constexpr int kMmaWarp = 8;
+constexpr int kMmaWarp = 8;    // MMA issue for subtile 0; owns the TMEM allocation
 constexpr int kTmaWarp = 9;
+constexpr int kMmaWarp1 = 10;  // MMA issue for subtile 1 when kMmaWarps == 2
+constexpr int kMmaWarps = 1;   // warps issuing MMAs: 1 (both subtiles) or 2 (one each)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 enum : int { MASK_NONE = 0, MASK_CAUSAL = 1, MASK_WINDOW = 2, MASK_DOCUMENT = 3 };
 enum : int { MOD_NONE = 0, MOD_SOFTCAP = 1, MOD_ALIBI = 2 };
-enum : int { DEV_TIMEOUT = 1, DEV_BAD_PAGE = 2, DEV_BAD_LEN = 4 };
+enum : int { DEV_TIMEOUT = 1, DEV_BAD_PAGE = 2, DEV_BAD_LEN = 4, DEV_BAD_MASK = 8 };
 
 struct FwdArgs {
   int B, Hq, Hkv, Sq, Skv, g;
@@ -78,8 +80,13 @@ struct FwdArgs {
   float scale;          // softmax scale
   int mask, wl, wr, q_offset;
   const int32_t* doc_id;
-  const uint8_t* bm_cls;  // [nQ][nK] class table or nullptr
+  int64_t doc_bstride;    // elements between the document rows of batches (0: one shared row)
+  const uint8_t* bm_cls;  // [Bm][Hm][nQ][nK] class tables or nullptr
   const int32_t *bm_part_cnt, *bm_part_idx, *bm_full_cnt, *bm_full_idx;  // ascending kv-tile lists
+  int bm_Bm, bm_Hm;       // slices of the block mask (1 = shared by every batch / head)
+  const int32_t* bm_row_order;   // [Bm][nQ] q-tiles heaviest first, or nullptr
+  const int32_t* bm_doc_start;   // [Bm][Sq] document run starts (document masks)
+  const int32_t* bm_doc_sorted;  // [Bm] 1: every document is one run of ids
   int nQ, nK;
   int mod;
   float softcap;
@@ -101,6 +108,10 @@ struct FwdArgs {
   float* part_o;    // [B][Hq][n_splits][D]
   float* part_lse;  // [B][Hq][n_splits]
   int* status;
+  // cycle trace (ATTN_TRACE builds only; null otherwise): per CTA and role,
+  // trace_per_role records of {cycles since kernel start, event << 24 | aux}
+  uint2* trace;
+  int trace_per_role;
 };
 
 template <int D, bool DECODE>
@@ -129,7 +140,8 @@ struct Barriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[6];
   uint64_t v_full[6];
-  uint64_t kv_empty[6];
+  uint64_t k_empty[6];    // the K tile of the slot has been read by every QK^T that uses it
+  uint64_t v_empty[6];    // the V tile of the slot has been read by every PV that uses it
   uint64_t s_ready[2];    // prefill: keys 0-63 of S ready (decode: the whole S)
   uint64_t p_ready[2];    // prefill: P for keys 0-63 written (decode: the whole P)
   uint64_t s_b_ready[2];  // prefill: keys 64-127 of S ready
@@ -138,10 +150,40 @@ struct Barriers {
   uint64_t o_done[2];
   uint64_t o_free[2];
   uint64_t merge_full, merge_empty;  // decode: subtile-1 row stats handed to subtile 0
-  uint64_t final_mma;
+  uint64_t final_mma[2];
+  uint64_t mma_turn[2];   // turn token between the two MMA warps (kMmaWarps == 2)
   uint32_t tmem_base;
   int abort_flag;
+  uint32_t trace_cnt[11]; // ATTN_TRACE: records written per role
+  long long trace_t0;     // ATTN_TRACE: clock64 at kernel start
 };
+
+// ---------------------------------------------------------------- cycle trace
+// Compiled in only with -DATTN_TRACE (a separate build of the library): lane
+// 0 of each role's warp (role = warp index: softmax warps 0-7, MMA warps 8 and
+// 10, TMA warp 9) appends {SM cycles since kernel start, event id << 24 | aux}
+// records to the caller's buffer. Normal builds contain none of this.
+enum : int {
+  kTraceRoles = 11, TR_TMA = 9,
+  EV_S_WAIT = 1, EV_S_READY = 2, EV_P_DONE = 3, EV_O_WAIT = 4, EV_EPI_BEGIN = 5, EV_EPI_END = 6,
+  EV_Q_FULL = 10, EV_PV = 11, EV_QK = 12, EV_P_WAIT = 13, EV_MMA_END = 14, EV_PV_ISSUED = 15,
+  EV_Q_LOAD = 20, EV_KV_LOAD = 21, EV_KERNEL_END = 30
+};
+#ifdef ATTN_TRACE
+__device__ __forceinline__ void trace_rec(const FwdArgs& a, Barriers& bar, int role, int ev, int aux) {
+  if ((threadIdx.x & 31) == 0 && a.trace != nullptr) {
+    const uint32_t n = bar.trace_cnt[role];
+    if (n < (uint32_t)a.trace_per_role) {
+      a.trace[((size_t)blockIdx.x * kTraceRoles + role) * a.trace_per_role + n] =
+          make_uint2((uint32_t)(clock64() - bar.trace_t0), ((uint32_t)ev << 24) | ((uint32_t)aux & 0xffffffu));
+      bar.trace_cnt[role] = n + 1;
+    }
+  }
+}
+#define ATTN_TRACE_REC(role, ev, aux) trace_rec(a, bar, (role), (ev), (aux))
+#else
+#define ATTN_TRACE_REC(role, ev, aux) ((void)0)
+#endif
 
 // ---------------------------------------------------------------- work map
 struct Work {
@@ -174,13 +216,20 @@ __device__ __forceinline__ Work map_work(const FwdArgs& a, int u) {
     w.t_begin = min(nt, w.split * a.tiles_per_split);
     w.t_end = min(nt, w.t_begin + a.tiles_per_split);
   } else {
-    // Heaviest row tiles first: unit index u walks row tiles from the end.
+    // Heaviest row tiles first: unit index u walks row tiles from the end
+    // (the causal and window forms), or in the block mask's work order.
     const int HU = a.pair_heads ? a.Hq / 2 : a.Hq;
     const int per = a.B * HU;
     const int qi = u / per, rem = u % per;
     w.b = rem / HU;
     const int hu = rem % HU;
-    const int rt = a.n_row_units - 1 - qi;
+    int rt = a.n_row_units - 1 - qi;
+    if (a.bm_row_order != nullptr && a.pair_heads) {
+      // a caller-written order entry outside the q-tiles falls back to the
+      // default order (the producer reports it as a bad mask)
+      const int o = __ldg(a.bm_row_order + (int64_t)(a.bm_Bm == 1 ? 0 : w.b) * a.nQ + qi);
+      if (o >= 0 && o < a.n_row_units) rt = o;
+    }
     if (a.pair_heads) {
       w.head0 = 2 * hu;
       w.head1 = 2 * hu + 1;
@@ -198,6 +247,11 @@ __device__ __forceinline__ Work map_work(const FwdArgs& a, int u) {
   return w;
 }
 
+// Block-mask slice (batch, head) that serves query head h of batch b.
+__device__ __forceinline__ int64_t bm_slice(const FwdArgs& a, int b, int h) {
+  return (int64_t)(a.bm_Bm == 1 ? 0 : b) * a.bm_Hm + (a.bm_Hm == 1 ? 0 : h);
+}
+
 // Tile class of kv tile t for subtile s: 0 empty, 1 partial, 2 full. BM:
 // the classes come from a block mask's table instead of the window bounds.
 template <bool DECODE, bool BM>
@@ -208,14 +262,14 @@ __device__ __forceinline__ int tile_class(const FwdArgs& a, const Work& w, int s
     return (t + 1) * kKeys <= w.seqlen ? 2 : 1;
   } else {
     const int r0 = w_row0(w, s);
-    if (r0 >= a.Sq || t >= a.nK) return 0;
+    if (r0 >= a.Sq || t < 0 || t >= a.nK) return 0;
     const int r1 = min(r0 + kRows, a.Sq) - 1;
     const int c0 = t * kKeys;
     const int c1 = min(c0 + kKeys, a.Skv) - 1;
     const bool ragged = c0 + kKeys > a.Skv;
     int cls;
     if constexpr (BM) {
-      cls = a.bm_cls[(r0 / kRows) * a.nK + t];
+      cls = a.bm_cls[(bm_slice(a, w.b, w_head(w, s)) * a.nQ + r0 / kRows) * a.nK + t];
     } else if (a.mask == MASK_NONE) {
       cls = 2;
     } else {
@@ -302,19 +356,22 @@ __device__ __forceinline__ int walker_init(const FwdArgs& a, const Work& w, Tile
     tw.t = lo;
     return hi - lo + 1;
   } else {
+    // row q-tile of each subtile within its (batch, head) slice; the second
+    // list is needed only when the subtiles differ in rows or in slice
+    const int64_t q0 = bm_slice(a, w.b, w.head0) * a.nQ + w.row00 / kRows;
+    const int64_t q1 = bm_slice(a, w.b, w.head1) * a.nQ + w.row01 / kRows;
+    // counts are clamped to a row's length, so lists are never read past it
     if (w.row00 < a.Sq) {
-      const int qt = w.row00 / kRows;
-      tw.np0 = __ldg(a.bm_part_cnt + qt);
-      tw.nf0 = __ldg(a.bm_full_cnt + qt);
-      tw.p0 = a.bm_part_idx + (int64_t)qt * a.nK;
-      tw.f0 = a.bm_full_idx + (int64_t)qt * a.nK;
+      tw.np0 = min(max(__ldg(a.bm_part_cnt + q0), 0), a.nK);
+      tw.nf0 = min(max(__ldg(a.bm_full_cnt + q0), 0), a.nK);
+      tw.p0 = a.bm_part_idx + q0 * a.nK;
+      tw.f0 = a.bm_full_idx + q0 * a.nK;
     }
-    if (w.row01 < a.Sq && w.row01 != w.row00) {
-      const int qt = w.row01 / kRows;
-      tw.np1 = __ldg(a.bm_part_cnt + qt);
-      tw.nf1 = __ldg(a.bm_full_cnt + qt);
-      tw.p1 = a.bm_part_idx + (int64_t)qt * a.nK;
-      tw.f1 = a.bm_full_idx + (int64_t)qt * a.nK;
+    if (w.row01 < a.Sq && q1 != q0) {
+      tw.np1 = min(max(__ldg(a.bm_part_cnt + q1), 0), a.nK);
+      tw.nf1 = min(max(__ldg(a.bm_full_cnt + q1), 0), a.nK);
+      tw.p1 = a.bm_part_idx + q1 * a.nK;
+      tw.f1 = a.bm_full_idx + q1 * a.nK;
     }
     // count the union, then rewind
     int n = 0;
@@ -340,13 +397,12 @@ __device__ __forceinline__ void walker_next(TileWalker& tw) {
 }
 
 // ---------------------------------------------------------------- producer
+// Loads key tile t of K or of V (map m) into dst, completing on bar.
 template <int D, bool DECODE>
-__device__ __forceinline__ void load_kv_tile(const FwdArgs& a, const Work& w, const CUtensorMap* mk,
-                                             const CUtensorMap* mv, uint8_t* kdst, uint8_t* vdst, uint64_t* kbar,
-                                             uint64_t* vbar, int t, bool absent) {
+__device__ __forceinline__ void load_kv_tile(const FwdArgs& a, const Work& w, const CUtensorMap* m, uint8_t* dst,
+                                             uint64_t* bar, int t, bool absent, bool report) {
   using L = Layout<D, DECODE>;
-  mbar_arrive_expect_tx(kbar, L::kTileBytes);
-  mbar_arrive_expect_tx(vbar, L::kTileBytes);
+  mbar_arrive_expect_tx(bar, L::kTileBytes);
   if constexpr (DECODE) {
     const int rows = a.box_rows;
     for (int u = 0; u < kKeys / rows; ++u) {
@@ -358,21 +414,16 @@ __device__ __forceinline__ void load_kv_tile(const FwdArgs& a, const Work& w, co
         const int pg = a.block_table[(int64_t)w.b * a.bt_stride + lp];
         if (pg >= 0 && pg < a.num_pages) {
           phys = pg;
-        } else if (a.status) {
+        } else if (a.status && report) {
           atomicOr(a.status, DEV_BAD_PAGE);
         }
       }
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_4d(kdst + c * L::kChunk + u * rows * 128, mk, kbar, c * 64, w.hk, slot, phys);
-        tma_load_4d(vdst + c * L::kChunk + u * rows * 128, mv, vbar, c * 64, w.hk, slot, phys);
-      }
+      for (int c = 0; c < D / 64; ++c) tma_load_4d(dst + c * L::kChunk + u * rows * 128, m, bar, c * 64, w.hk, slot, phys);
     }
   } else {
     (void)absent;
-    for (int c = 0; c < D / 64; ++c) {
-      tma_load_4d(kdst + c * L::kChunk, mk, kbar, c * 64, t * kKeys, w.hk, w.b);
-      tma_load_4d(vdst + c * L::kChunk, mv, vbar, c * 64, t * kKeys, w.hk, w.b);
-    }
+    (void)report;
+    for (int c = 0; c < D / 64; ++c) tma_load_4d(dst + c * L::kChunk, m, bar, c * 64, t * kKeys, w.hk, w.b);
   }
 }
 
@@ -492,7 +543,9 @@ struct MaskRow {
   int clo;
   unsigned span;  // 0xffffffff sentinel handled by 'none'
   bool none;
-  int dq;         // document id of the query row (document mask)
+  bool by_id;     // document mask with unsorted ids: compare ids per key
+  int dq;         // document id of the query row (by_id)
+  const int32_t* doc;  // document ids of this batch (by_id)
 };
 
 template <bool DECODE, bool BM>
@@ -501,6 +554,8 @@ __device__ __forceinline__ MaskRow mask_row(const FwdArgs& a, const Work& w, int
   const int kv0 = t * kKeys;
   long lo, hi;
   m.dq = 0;
+  m.doc = a.doc_id;
+  m.by_id = false;
   if constexpr (DECODE) {
     lo = 0;
     hi = (long)w.seqlen - 1;
@@ -508,9 +563,18 @@ __device__ __forceinline__ MaskRow mask_row(const FwdArgs& a, const Work& w, int
     const int qrow = w_row0(w, s) + row;
     const long q_pos = (long)qrow + a.q_offset;
     if (BM && a.mask == MASK_DOCUMENT) {
-      lo = 0;
+      // Sorted ids: the row's keys are the interval [start of its run, q]
+      // and take the range path; otherwise ids are compared key by key.
+      const int bs = a.bm_Bm == 1 ? 0 : w.b;
       hi = q_pos;
-      m.dq = a.doc_id[min(qrow, a.Sq - 1)];
+      if (__ldg(a.bm_doc_sorted + bs)) {
+        lo = __ldg(a.bm_doc_start + (int64_t)bs * a.Sq + min(qrow, a.Sq - 1));
+      } else {
+        lo = 0;
+        m.by_id = true;
+        m.doc = a.doc_id + (int64_t)w.b * a.doc_bstride;
+        m.dq = m.doc[min(qrow, a.Sq - 1)];
+      }
     } else {
       lo = a.wl >= 0 ? q_pos - a.wl : -(1l << 40);
       hi = a.wr >= 0 ? q_pos + a.wr : (1l << 40);
@@ -536,9 +600,9 @@ __device__ __forceinline__ MaskRow mask_row(const FwdArgs& a, const Work& w, int
 template <bool DECODE, bool BM>
 __device__ __forceinline__ bool mask_chunk(const FwdArgs& a, const MaskRow& m, int t, int c, float* x) {
   const float NEG_INF = -__int_as_float(0x7f800000);
-  if (BM && a.mask == MASK_DOCUMENT) {
+  if (BM && a.mask == MASK_DOCUMENT && m.by_id) {
     const int kv = t * kKeys + 32 * c;
-    const int4* d4 = reinterpret_cast<const int4*>(a.doc_id + kv);
+    const int4* d4 = reinterpret_cast<const int4*>(m.doc + kv);
     // keys of this chunk inside the sequence: whole groups of four are read
     // as one 16-byte load, a ragged last group (Skv not a multiple of 4)
     // element by element; keys past Skv fail the span test below anyway.
@@ -554,7 +618,7 @@ __device__ __forceinline__ bool mask_chunk(const FwdArgs& a, const MaskRow& m, i
                      : "=r"(d.x), "=r"(d.y), "=r"(d.z), "=r"(d.w)
                      : "l"(d4 + i4));
       } else if (i4 == n4 && tail > 0) {
-        const int32_t* dp = a.doc_id + kv + 4 * i4;
+        const int32_t* dp = m.doc + kv + 4 * i4;
         d.x = __ldg(dp);
         if (tail > 1) d.y = __ldg(dp + 1);
         if (tail > 2) d.z = __ldg(dp + 2);
@@ -629,12 +693,15 @@ __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, in
   MaskRow mr;
   if constexpr (MASKED) mr = mask_row<DECODE, BM>(a, w, s, row, t);
   float mc = NEG_INF;
-  tmem_ld32f(tS, x);
+  // All four chunks are requested before a single wait: one exposed TMEM
+  // load latency per tile instead of one per chunk (measured 2.5 % faster
+  // on the causal prefill than keeping one chunk in flight).
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32f(tS + 32 * c, x + 32 * c);
   tmem_ld_wait();
-  reg_fence_f<32>(x);
+  reg_fence_f<128>(x);
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    if (c < 3) tmem_ld32f(tS + 32 * (c + 1), x + 32 * (c + 1));
     if constexpr (MOD != MOD_NONE) mod_chunk<DECODE, MOD>(a, w, s, row, t, c, x + 32 * c);
     bool dead = false;
     if constexpr (MASKED) dead = mask_chunk<DECODE, BM>(a, mr, t, c, x + 32 * c);
@@ -653,10 +720,6 @@ __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, in
       exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
     }
     tmem_st16(tS + 16 * c, pk);
-    if (c < 3) {
-      tmem_ld_wait();
-      reg_fence_f<32>(x + 32 * (c + 1));
-    }
   }
   return mc;
 }
@@ -671,19 +734,15 @@ __device__ __forceinline__ float prepare_tile(const FwdArgs& a, const Work& w, i
   MaskRow mr;
   if constexpr (MASKED) mr = mask_row<DECODE, BM>(a, w, s, row, t);
   float mc = NEG_INF;
-  tmem_ld32f(tS, x);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32f(tS + 32 * c, x + 32 * c);
   tmem_ld_wait();
-  reg_fence_f<32>(x);
+  reg_fence_f<128>(x);
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    if (c < 3) tmem_ld32f(tS + 32 * (c + 1), x + 32 * (c + 1));
     if constexpr (MOD != MOD_NONE) mod_chunk<DECODE, MOD>(a, w, s, row, t, c, x + 32 * c);
     if constexpr (MASKED) (void)mask_chunk<DECODE, BM>(a, mr, t, c, x + 32 * c);
     mc = fmaxf(mc, chunk_max(x + 32 * c));
-    if (c < 3) {
-      tmem_ld_wait();
-      reg_fence_f<32>(x + 32 * (c + 1));
-    }
   }
   return mc;
 }
@@ -834,12 +893,12 @@ __device__ __forceinline__ float stream_half(const FwdArgs& a, const Work& w, in
   float mc = NEG_INF;
   const uint32_t base = tS + 64 * h;
   tmem_ld32f(base, x);
+  tmem_ld32f(base + 32, x + 32);
   tmem_ld_wait();
-  reg_fence_f<32>(x);
+  reg_fence_f<64>(x);
 #pragma unroll
   for (int cc = 0; cc < 2; ++cc) {
     const int c = 2 * h + cc;
-    if (cc == 0) tmem_ld32f(base + 32, x + 32);
     if constexpr (MOD != MOD_NONE) mod_chunk<false, MOD>(a, w, s, row, t, c, x + 32 * cc);
     bool dead = false;
     if constexpr (MASKED) dead = mask_chunk<false, BM>(a, mr, t, c, x + 32 * cc);
@@ -857,10 +916,6 @@ __device__ __forceinline__ float stream_half(const FwdArgs& a, const Work& w, in
       exp_chunk(x + 32 * cc, MULT, NMU, pk, acc0, acc1);
     }
     tmem_st16(base + 16 * cc, pk);
-    if (cc == 0) {
-      tmem_ld_wait();
-      reg_fence_f<32>(x + 32);
-    }
   }
   return mc;
 }
@@ -876,19 +931,15 @@ __device__ __forceinline__ float prepare_half(const FwdArgs& a, const Work& w, i
   float mc = NEG_INF;
   const uint32_t base = tS + 64 * h;
   tmem_ld32f(base, x);
+  tmem_ld32f(base + 32, x + 32);
   tmem_ld_wait();
-  reg_fence_f<32>(x);
+  reg_fence_f<64>(x);
 #pragma unroll
   for (int cc = 0; cc < 2; ++cc) {
     const int c = 2 * h + cc;
-    if (cc == 0) tmem_ld32f(base + 32, x + 32);
     if constexpr (MOD != MOD_NONE) mod_chunk<false, MOD>(a, w, s, row, t, c, x + 32 * cc);
     if constexpr (MASKED) (void)mask_chunk<false, BM>(a, mr, t, c, x + 32 * cc);
     mc = fmaxf(mc, chunk_max(x + 32 * cc));
-    if (cc == 0) {
-      tmem_ld_wait();
-      reg_fence_f<32>(x + 32);
-    }
   }
   return mc;
 }
@@ -1151,7 +1202,7 @@ __device__ __forceinline__ bool epilogue(const FwdArgs& a, const CUtensorMap* ma
 // K/V ring across units. Barrier phases count events across units:
 //   q_full / q_empty / o_done / o_free   once per unit that has key tiles,
 //   s_ready / p_ready                     once per step,
-//   k_full / v_full / kv_empty            once per K/V load.
+//   k_full / v_full / k_empty / v_empty   once per K/V load.
 // While the softmax warps write a unit's outputs, the producer already loads
 // the next unit's Q and K/V and the MMA warp runs its first QK^T products.
 template <int D, bool DECODE, int MOD, bool BM>
@@ -1170,12 +1221,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     bar.abort_flag = 0;
+#ifdef ATTN_TRACE
+    bar.trace_t0 = clock64();
+    for (int r = 0; r < kTraceRoles; ++r) bar.trace_cnt[r] = 0;
+#endif
     mbar_init(&bar.q_full, 1);
-    mbar_init(&bar.q_empty, 1);
+    mbar_init(&bar.q_empty, 2);  // the last QK^T of each subtile's MMA warp
     for (int i = 0; i < L::kNSlot; ++i) {
       mbar_init(&bar.k_full[i], 1);
       mbar_init(&bar.v_full[i], 1);
-      mbar_init(&bar.kv_empty[i], 1);
+      // prefill: both subtiles read every K/V tile; decode: one subtile does
+      mbar_init(&bar.k_empty[i], DECODE ? 1 : 2);
+      mbar_init(&bar.v_empty[i], DECODE ? 1 : 2);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar.s_ready[s], 1);
@@ -1188,7 +1245,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bar.merge_full, 128);
     mbar_init(&bar.merge_empty, 128);
-    mbar_init(&bar.final_mma, 1);
+    mbar_init(&bar.final_mma[0], 1);
+    mbar_init(&bar.final_mma[1], 1);
+    mbar_init(&bar.mma_turn[0], 1);
+    mbar_init(&bar.mma_turn[1], 1);
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -1226,7 +1286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&map_v);
     }
     __syncwarp();
-    int kload = 0;  // K/V loads issued so far: ring position and phase
+    int kload = 0;  // K/V tile pairs started so far: ring position and phase
+    int vload = 0;  // V tiles issued so far (one behind kload while a pair is half issued)
     int qcnt = 0;   // units with key tiles so far
     bool ok = true;
     for (int r = 0; ok && r < rounds; ++r) {
@@ -1240,6 +1301,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           atomicOr(a.status, DEV_BAD_LEN);
         __syncwarp();
       }
+      if constexpr (BM) {
+        // caller-written tables: an order entry outside the q-tiles, or a
+        // count outside [0, n_kv_tiles], is reported (and was not followed)
+        const int qi = u / (a.B * (a.pair_heads ? a.Hq / 2 : a.Hq));
+        bool bad = false;
+        if (a.bm_row_order != nullptr && a.pair_heads) {
+          const int o = __ldg(a.bm_row_order + (int64_t)(a.bm_Bm == 1 ? 0 : w.b) * a.nQ + qi);
+          bad = o < 0 || o >= a.n_row_units;
+        }
+        for (int s = 0; s < 2; ++s) {
+          if (w_row0(w, s) >= a.Sq) continue;
+          const int64_t q = bm_slice(a, w.b, w_head(w, s)) * a.nQ + w_row0(w, s) / kRows;
+          const int pc = __ldg(a.bm_part_cnt + q), fc = __ldg(a.bm_full_cnt + q);
+          bad |= pc < 0 || pc > a.nK || fc < 0 || fc > a.nK;
+        }
+        if (bad && a.status && elect_one_sync()) atomicOr(a.status, DEV_BAD_MASK);
+        __syncwarp();
+      }
       TileWalker tw;
       const int n = walker_init<DECODE, BM>(a, w, tw);
       if (n == 0) continue;
@@ -1247,6 +1326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
+      ATTN_TRACE_REC(TR_TMA, EV_Q_LOAD, qcnt);
       if (elect_one_sync()) {
         mbar_arrive_expect_tx(&bar.q_full, L::kNQ * L::kTileBytes);
         for (int s = 0; s < L::kNQ; ++s)
@@ -1259,23 +1339,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
       }
       __syncwarp();
+      if constexpr (!DECODE) {
+        // Q is read once per unit, so the next unit's Q would come from HBM
+        // while its first QK^T waits: pull it into L2 now, a unit ahead.
+        const int un = r + 1 < rounds ? unit_of(r + 1) : -1;
+        if (un >= 0) {
+          const Work wn = map_work<DECODE>(a, un);
+          if (elect_one_sync()) {
+            for (int s = 0; s < 2; ++s)
+              if (w_row0(wn, s) < a.Sq)
+                for (int c = 0; c < D / 64; ++c) tma_prefetch_l2_4d(&map_q, c * 64, w_row0(wn, s), w_head(wn, s), wn.b);
+          }
+          __syncwarp();
+        }
+      }
       ++qcnt;
       const int n_loads = DECODE ? 2 * n : n;
       for (int k = 0; k < n_loads; ++k) {
         const int t = tw.t;
         const int slot = kload % L::kNSlot;
         const int use = kload / L::kNSlot;
-        if (use > 0 && !wait_all(&bar.kv_empty[slot], (use - 1) & 1)) {
+        const bool absent = DECODE && t >= w.t_end;
+        // K and V of a slot are released separately (K once its last QK^T has
+        // read it, V after its last PV), so the next K can land a step earlier.
+        if (use > 0 && !wait_all(&bar.k_empty[slot], (use - 1) & 1)) {
           ok = false;
           break;
         }
-        const bool absent = DECODE && t >= w.t_end;
+        ATTN_TRACE_REC(TR_TMA, EV_KV_LOAD, kload);
         if (elect_one_sync())
-          load_kv_tile<D, DECODE>(a, w, &map_k, &map_v, smem + L::kKOff + slot * L::kTileBytes,
-                                  smem + L::kVOff + slot * L::kTileBytes, &bar.k_full[slot], &bar.v_full[slot], t,
-                                  absent);
+          load_kv_tile<D, DECODE>(a, w, &map_k, smem + L::kKOff + slot * L::kTileBytes, &bar.k_full[slot], t, absent,
+                                  true);
         __syncwarp();
         ++kload;
+        if (use > 0 && !wait_all(&bar.v_empty[slot], (use - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        if (elect_one_sync())
+          load_kv_tile<D, DECODE>(a, w, &map_v, smem + L::kVOff + slot * L::kTileBytes, &bar.v_full[slot], t, absent,
+                                  false);
+        __syncwarp();
+        ++vload;
         if (DECODE)
           ++tw.t;
         else
@@ -1285,17 +1390,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Drain: on an abort, wait (bounded) for every copy still in flight so
     // none lands in shared memory after the CTA has exited.
     if (*abort_flag) {
-      for (int k = max(0, kload - L::kNSlot); k < kload; ++k) {
-        const int slot = k % L::kNSlot;
-        const uint32_t par = (k / L::kNSlot) & 1;
-        mbar_wait_timeout(&bar.k_full[slot], par);
-        mbar_wait_timeout(&bar.v_full[slot], par);
-      }
+      for (int k = max(0, kload - L::kNSlot); k < kload; ++k)
+        mbar_wait_timeout(&bar.k_full[k % L::kNSlot], (k / L::kNSlot) & 1);
+      for (int k = max(0, vload - L::kNSlot); k < vload; ++k)
+        mbar_wait_timeout(&bar.v_full[k % L::kNSlot], (k / L::kNSlot) & 1);
       if (qcnt > 0) mbar_wait_timeout(&bar.q_full, (qcnt - 1) & 1);
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarp || (kMmaWarps == 2 && warp == kMmaWarp1)) {
     regs_decrease<kControlRegs>();
     // ------------------------------------------------------------ MMA issue
+    // A thread that issues tcgen05.mma stalls until the tensor pipe accepts
+    // the MMA, so every wait and fence between two batches of MMAs leaves the
+    // pipe idle: a step's PV and the next QK^T of a subtile therefore go out
+    // back to back from one elected lane. The subtiles take turns in a fixed
+    // order (PV(0) QK(0) PV(1) QK(1) per step), which keeps the ping-pong:
+    // one subtile's softmax runs while the other's MMAs execute.
+    // With kMmaWarps == 2 each subtile has its own issuing warp and the two
+    // hand a turn token to each other, so one warp's waits overlap the other
+    // warp's batch.
+    constexpr int kSubPerWarp = kMmaWarps == 2 ? 1 : 2;
+    const int s_first = (kMmaWarps == 2 && warp == kMmaWarp1) ? 1 : 0;
+    const int trole = warp;
+    (void)trole;
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kKeys, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
     // Descriptor low words (start address in 16-byte units + LBO); every
@@ -1305,20 +1421,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t k_lo = sdesc_sw128_lo(smem_u32(smem + L::kKOff), 16);
     const uint32_t v_lo = sdesc_sw128_lo(smem_u32(smem + L::kVOff), L::kChunk);
     constexpr uint32_t kTileUnits = L::kTileBytes >> 4;
-    // last: the unit's final QK^T of subtile 1, after which Q may be reloaded.
-    auto issue_qk = [&](int s, int slot, bool last) {
+    // QK^T of subtile s into S(s) (elected lane only). last: the unit's
+    // final QK^T of s, after which (once both subtiles' are done) Q may be
+    // reloaded. The K tile of the slot is released once every subtile that
+    // reads it has issued its QK^T.
+    auto qk_mmas = [&](int s, int slot, bool last) {
       const uint32_t qa = q_lo + (DECODE ? 0u : (uint32_t)s * kTileUnits);
       const uint32_t ka = k_lo + (uint32_t)slot * kTileUnits;
-      if (elect_one_sync()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
-          mma_ss(tmem + s * 128, sdesc_join(qa + off, kHi), sdesc_join(ka + off, kHi), idesc_qk, kk > 0);
-        }
-        mma_commit(&bar.s_ready[s]);
-        if (last) mma_commit(&bar.q_empty);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
+        mma_ss(tmem + s * 128, sdesc_join(qa + off, kHi), sdesc_join(ka + off, kHi), idesc_qk, kk > 0);
       }
-      __syncwarp();
+      mma_commit(&bar.s_ready[s]);
+      if (last) mma_commit(&bar.q_empty);
+      mma_commit(&bar.k_empty[slot]);
+    };
+    // Prefill with a score mod: QK^T and PV in key halves (see "prefill, half tiles").
+    constexpr uint32_t idesc_qk_half = idesc_bf16_f32(128, 64, 0, 0);
+    constexpr uint32_t kHalfKeyUnits = (64 * 128) >> 4;  // 64 K rows of a 128-byte SW128 box
+    auto qk_half_mmas = [&](int s, int slot, int h, bool last) {
+      const uint32_t qa = q_lo + (uint32_t)s * kTileUnits;
+      const uint32_t ka = k_lo + (uint32_t)slot * kTileUnits + (uint32_t)h * kHalfKeyUnits;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
+        mma_ss(tmem + s * 128 + 64 * h, sdesc_join(qa + off, kHi), sdesc_join(ka + off, kHi), idesc_qk_half, kk > 0);
+      }
+      mma_commit(h == 0 ? &bar.s_ready[s] : &bar.s_b_ready[s]);
+      if (last) mma_commit(&bar.q_empty);
+      if (h == 1) mma_commit(&bar.k_empty[slot]);
     };
     auto slot_of = [&](int g, int s) { return DECODE ? (2 * g + s) % L::kNSlot : g % L::kNSlot; };
     auto phase_of = [&](int g, int s) { return (uint32_t)(((DECODE ? 2 * g + s : g) / L::kNSlot) & 1); };
@@ -1334,68 +1466,76 @@ __global__ void __launch_bounds__(kThreads, 1)
       TileWalker tw;
       return walker_init<DECODE, BM>(a, w, tw);
     };
+    // Turn token between two issuing warps: batch b of subtile 1 follows
+    // batch b of subtile 0, batch b + 1 of subtile 0 follows batch b of
+    // subtile 1 (one arrival each; phases count batches).
+    int batch = 0;
+    auto take_turn = [&](int s) -> bool {
+      if constexpr (kMmaWarps == 2) {
+        if (s == 1) return wait_spin_all(&bar.mma_turn[1], batch & 1);
+        if (batch > 0) return wait_spin_all(&bar.mma_turn[0], (batch - 1) & 1);
+      }
+      (void)s;
+      return true;
+    };
+    auto pass_turn = [&](int s) {
+      if constexpr (kMmaWarps == 2) {
+        if (elect_one_sync()) mbar_arrive(&bar.mma_turn[s ^ 1]);
+        __syncwarp();
+      }
+      (void)s;
+    };
     int gstep = 0;  // steps issued so far across units
     int qcnt = 0;   // units with key tiles so far
     bool ok = true;
-    // Prefill: QK^T and PV in key halves (see "prefill, half tiles").
-    constexpr uint32_t idesc_qk_half = idesc_bf16_f32(128, 64, 0, 0);
-    constexpr uint32_t kHalfKeyUnits = (64 * 128) >> 4;  // 64 K rows of a 128-byte SW128 box
-    auto issue_qk_half = [&](int s, int slot, int h, uint64_t* done, bool last) {
-      const uint32_t qa = q_lo + (uint32_t)s * kTileUnits;
-      const uint32_t ka = k_lo + (uint32_t)slot * kTileUnits + (uint32_t)h * kHalfKeyUnits;
-      if (elect_one_sync()) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
-          mma_ss(tmem + s * 128 + 64 * h, sdesc_join(qa + off, kHi), sdesc_join(ka + off, kHi), idesc_qk_half,
-                 kk > 0);
-        }
-        mma_commit(done);
-        if (last) mma_commit(&bar.q_empty);
-      }
-      __syncwarp();
-    };
     int n_next = unit_steps(0);
     for (int r = 0; ok && r < rounds; ++r) {
       const int n = n_next;
       if (n > 0) {
         ok = wait_all(&bar.q_full, qcnt & 1);
-        if (ok) ok = wait_all(&bar.k_full[slot_of(gstep, 0)], phase_of(gstep, 0));
-        if (ok) {
+        ATTN_TRACE_REC(trole, EV_Q_FULL, qcnt);
+#pragma unroll
+        for (int si = 0; si < kSubPerWarp && ok; ++si) {
+          const int s = s_first + si;
+          ok = wait_all(&bar.k_full[slot_of(gstep, s)], phase_of(gstep, s));
+          if (!ok) break;
           tc_fence_after();
-          if constexpr (!kHalfTiles<DECODE, MOD>) {
-            issue_qk(0, slot_of(gstep, 0), false);
-            if (DECODE) ok = wait_all(&bar.k_full[slot_of(gstep, 1)], phase_of(gstep, 1));
-            tc_fence_after();
-            if (ok) issue_qk(1, slot_of(gstep, 1), n == 1);
-          } else {
-            const int slot = slot_of(gstep, 0);
-            issue_qk_half(0, slot, 0, &bar.s_ready[0], false);
-            issue_qk_half(1, slot, 0, &bar.s_ready[1], false);
-            issue_qk_half(0, slot, 1, &bar.s_b_ready[0], false);
-            issue_qk_half(1, slot, 1, &bar.s_b_ready[1], n == 1);
+          if (elect_one_sync()) {
+            if constexpr (!kHalfTiles<DECODE, MOD>) {
+              qk_mmas(s, slot_of(gstep, s), n == 1);
+            } else {
+              qk_half_mmas(s, slot_of(gstep, s), 0, false);
+              qk_half_mmas(s, slot_of(gstep, s), 1, n == 1);
+            }
           }
+          __syncwarp();
         }
       }
       n_next = unit_steps(r + 1);
       if (n == 0) continue;
-      if constexpr (kHalfTiles<DECODE, MOD>) {
-        for (int j = 0; ok && j < n; ++j) {
-          const int g = gstep + j;
-          const bool more = j + 1 < n;
-          const int slot = slot_of(g, 0);
-          const int nslot = slot_of(g + 1, 0);
-          if (!wait_all(&bar.v_full[slot], phase_of(g, 0))) { ok = false; break; }
-          const uint32_t va = v_lo + (uint32_t)slot * kTileUnits;
+      for (int j = 0; ok && j < n; ++j) {
+        const int g = gstep + j;
+        const bool more = j + 1 < n;
+        constexpr int kHalves = kHalfTiles<DECODE, MOD> ? 2 : 1;
 #pragma unroll
-          for (int h = 0; h < 2 && ok; ++h) {
+        for (int h = 0; h < kHalves && ok; ++h) {
 #pragma unroll
-            for (int s = 0; s < 2; ++s) {
-              if (!wait_spin_all(h == 0 ? &bar.p_ready[s] : &bar.p_b_ready[s], g & 1)) { ok = false; break; }
-              // The first PV of a unit overwrites O(s): the previous unit's epilogue must have read it.
-              if (j == 0 && h == 0 && qcnt > 0 && !wait_all(&bar.o_free[s], (qcnt - 1) & 1)) { ok = false; break; }
-              tc_fence_after();
-              if (elect_one_sync()) {
+          for (int si = 0; si < kSubPerWarp; ++si) {
+            const int s = s_first + si;
+            const int slot = slot_of(g, s), nslot = slot_of(g + 1, s);
+            const uint32_t va = v_lo + (uint32_t)slot * kTileUnits;
+            if (h == 0 && !wait_all(&bar.v_full[slot], phase_of(g, s))) { ok = false; break; }
+            if (h == 0 && more && !wait_all(&bar.k_full[nslot], phase_of(g + 1, s))) { ok = false; break; }
+            ATTN_TRACE_REC(trole, EV_P_WAIT, (g << 1) | s);
+            uint64_t* pbar = h == 0 ? &bar.p_ready[s] : &bar.p_b_ready[s];
+            if (!wait_spin_all(pbar, g & 1)) { ok = false; break; }
+            // The first PV of a unit overwrites O(s): the previous unit's epilogue must have read it.
+            if (j == 0 && h == 0 && qcnt > 0 && !wait_all(&bar.o_free[s], (qcnt - 1) & 1)) { ok = false; break; }
+            if (!take_turn(s)) { ok = false; break; }
+            tc_fence_after();
+            ATTN_TRACE_REC(trole, EV_PV, (g << 1) | s);
+            if (elect_one_sync()) {
+              if constexpr (kHalfTiles<DECODE, MOD>) {
                 // PV over keys 64h..64h+63: P from S(s) columns [64h, 64h+32), V rows 64h..
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
@@ -1404,58 +1544,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                          (j == 0 && h == 0 && kk == 0) ? 0u : 1u);
                 if (h == 0) mma_commit(&bar.pv_a_done[s]);
                 if (h == 1 && !more) mma_commit(&bar.o_done[s]);
-                if (h == 1 && s == 1) mma_commit(&bar.kv_empty[slot]);
-              }
-              __syncwarp();
-              if (more) {
-                if (h == 0 && s == 0 && !wait_all(&bar.k_full[nslot], phase_of(g + 1, 0))) { ok = false; break; }
-                tc_fence_after();
-                issue_qk_half(s, nslot, h, h == 0 ? &bar.s_ready[s] : &bar.s_b_ready[s],
-                              h == 1 && s == 1 && j + 2 == n);
+                if (h == 1) mma_commit(&bar.v_empty[slot]);
+                if (more) qk_half_mmas(s, nslot, h, h == 1 && j + 2 == n);
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < kKeys / 16; ++kk)
+                  mma_ts(tmem + 256 + s * L::kOCols, tmem + s * 128 + kk * 8,
+                         sdesc_join(va + ((kk * 16 * 128) >> 4), kHi), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                if (!more) mma_commit(&bar.o_done[s]);
+                mma_commit(&bar.v_empty[slot]);
+                if (more) qk_mmas(s, nslot, j + 2 == n);
               }
             }
+            __syncwarp();
+            pass_turn(s);
+            ++batch;
+            ATTN_TRACE_REC(trole, EV_PV_ISSUED, (g << 1) | s);
           }
         }
-      } else {
-      for (int j = 0; ok && j < n; ++j) {
-        const int g = gstep + j;
-        const bool more = j + 1 < n;
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          const int slot = slot_of(g, s);
-          if (!wait_all(&bar.v_full[slot], phase_of(g, s))) { ok = false; break; }
-          if (!wait_spin_all(&bar.p_ready[s], g & 1)) { ok = false; break; }
-          // The first PV of a unit overwrites O(s): the previous unit's epilogue must have read it.
-          if (j == 0 && qcnt > 0 && !wait_all(&bar.o_free[s], (qcnt - 1) & 1)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t va = v_lo + (uint32_t)slot * kTileUnits;
-          if (elect_one_sync()) {
-#pragma unroll
-            for (int kk = 0; kk < kKeys / 16; ++kk)
-              mma_ts(tmem + 256 + s * L::kOCols, tmem + s * 128 + kk * 8,
-                     sdesc_join(va + ((kk * 16 * 128) >> 4), kHi), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-            if (!more) mma_commit(&bar.o_done[s]);
-            if (DECODE || s == 1) mma_commit(&bar.kv_empty[slot]);
-          }
-          __syncwarp();
-          if (more) {
-            const int nslot = slot_of(g + 1, s);
-            if (!wait_all(&bar.k_full[nslot], phase_of(g + 1, s))) { ok = false; break; }
-            tc_fence_after();
-            issue_qk(s, nslot, s == 1 && j + 2 == n);
-          }
-        }
-      }
       }
       gstep += n;
       ++qcnt;
     }
-    // Every MMA must be complete before TMEM is released.
-    if (elect_one_sync()) mma_commit(&bar.final_mma);
+    ATTN_TRACE_REC(trole, EV_MMA_END, gstep);
+    // Every MMA of this warp must be complete before TMEM is released.
+    if (elect_one_sync()) mma_commit(&bar.final_mma[s_first]);
     __syncwarp();
-    mbar_wait_timeout(&bar.final_mma, 0);
-  } else if (warp >= 10) {
-    regs_decrease<kControlRegs>();
+    mbar_wait_timeout(&bar.final_mma[s_first], 0);
+  } else if (warp >= kMmaWarp) {
+    regs_decrease<kControlRegs>();  // idle: completes the third warpgroup
   } else {
     regs_increase<kSoftmaxRegs>();
     // ------------------------------------------------------------ softmax
@@ -1493,8 +1610,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j) {
         const int t = tw.t;
         const int cls = tile_class<DECODE, BM>(a, w, s, t);
+        ATTN_TRACE_REC(warp, EV_S_WAIT, gstep + j);
         if (!wait_spin_all(&bar.s_ready[s], (gstep + j) & 1)) { ok = false; break; }
         tc_fence_after();
+        ATTN_TRACE_REC(warp, EV_S_READY, (gstep + j) | (cls << 20));
         if constexpr (!kHalfTiles<DECODE, MOD>) {
           softmax_step<D, DECODE, MOD, BM>(a, w, s, row, t, cls, tS, tO, j == 0, st, &bar.p_ready[s]);
         } else if (!softmax_step_halves<D, MOD, BM>(a, w, s, row, t, cls, tS, tO, j == 0, st, bar, gstep + j,
@@ -1502,6 +1621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
+        ATTN_TRACE_REC(warp, EV_P_DONE, gstep + j);
         if (DECODE)
           tw.t += 2;
         else
@@ -1510,14 +1630,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       setup(r + 1);
       if (!have_unit) continue;
+      ATTN_TRACE_REC(warp, EV_O_WAIT, qcnt);
       if (n > 0) {
         bool got = wait_all(&bar.o_done[s], qcnt & 1);
         if (DECODE && s == 0) got = got && wait_all(&bar.o_done[1], qcnt & 1);
         if (!got) break;
         tc_fence_after();
       }
+      ATTN_TRACE_REC(warp, EV_EPI_BEGIN, qcnt);
       // A unit without key tiles still writes its (all-masked) outputs.
       if (!epilogue<D, DECODE>(a, &map_o, w, s, row, lane_base, n > 0, st, extra, bar, qcnt, abort_flag)) break;
+      ATTN_TRACE_REC(warp, EV_EPI_END, qcnt);
       if (n == 0) continue;
       // O is read: the next unit's first PV may overwrite it. In decode the
       // subtile-0 threads read both accumulators and release both.
@@ -1544,6 +1667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, 512);
   }
   if (threadIdx.x == 0 && bar.abort_flag && a.status) atomicOr(a.status, DEV_TIMEOUT);
+  if (threadIdx.x == 0) ATTN_TRACE_REC(0, EV_KERNEL_END, 0);
 }
 
 }  // namespace attn_kernels

@@ -49,6 +49,9 @@ typedef enum {
 /* Bits the kernels OR into *status. */
 #define ATTN_DEV_TIMEOUT 1   /* a bounded pipeline wait gave up; outputs invalid */
 #define ATTN_DEV_BAD_PAGE 2  /* a block_table entry was outside [0, num_pages) */
+#define ATTN_DEV_BAD_MASK 8  /* prefill: a caller-written block-mask table had a row_order entry
+                                outside [0, n_q_tiles) or a count outside [0, n_kv_tiles); the
+                                entry was not followed (default order / clamped count) */
 #define ATTN_DEV_BAD_LEN 4   /* decode: a cache_seqlens[b] was negative or above max_seqlen;
                                 that sequence was computed over its first max_seqlen keys
                                 (none if negative) and its outputs are not the requested ones */
@@ -59,7 +62,7 @@ typedef enum {
  *   NONE      every key allowed
  *   CAUSAL    j <= q_pos                                   (q_idx >= kv_idx)
  *   WINDOW    (left < 0 || q_pos - j <= left) && (right < 0 || j - q_pos <= right)
- *   DOCUMENT  j <= q_pos && doc_id[i] == doc_id[j]   (packed sequences; Sq == Skv,
+ *   DOCUMENT  j <= q_pos && doc[b][i] == doc[b][j]   (packed sequences; Sq == Skv,
  *             q_offset == 0; needs a block mask built from the same spec) */
 typedef enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_WINDOW = 2, ATTN_MASK_DOCUMENT = 3 } attn_mask_kind;
 
@@ -74,35 +77,61 @@ typedef struct {
   int window_left;        /* WINDOW: keys at most this far behind; -1 = unbounded */
   int window_right;       /* WINDOW: keys at most this far ahead;  -1 = unbounded */
   int q_offset;           /* position of query 0 on the key axis (CAUSAL / WINDOW) */
-  const int32_t *doc_id;  /* DOCUMENT: device int32 [S] document id per position, 16-byte aligned */
+  const int32_t *doc_id;  /* DOCUMENT: device int32 document id per position, 16-byte aligned:
+                             row b (batch b) starts at doc_id + b * doc_batch_stride */
+  int64_t doc_batch_stride; /* elements between the rows of doc_id (a multiple of 4); 0 = one
+                               [S] row shared by every batch */
 } attn_mask_spec;
 
-/* Block mask (FlexAttention create_block_mask equivalent): per (q-tile,
+/* Block mask (FlexAttention create_block_mask(mask_mod, B, H, Q_LEN, KV_LEN,
+ * BLOCK_SIZE) equivalent, attention-gym issue 101): per (batch, head, q-tile,
  * kv-tile) class 0 = empty (skipped), 1 = partial (mask evaluated per
- * element), 2 = full (no mask work), and per q-tile the ascending kv-tile
- * lists of partial and full tiles. Broadcast over batch and heads. All arrays
- * live inside one caller-owned device buffer laid out by attn_block_mask_layout. */
+ * element), 2 = full (no mask work), and per (batch, head, q-tile) the
+ * ascending kv-tile lists of partial and full tiles. Bm / Hm are the batch and
+ * head extents of the tables: 1 means one slice shared by every batch / head,
+ * otherwise they equal the B / Hq of the forward call (slice (b, h) serves
+ * batch b, query head h). All arrays live inside one caller-owned device
+ * buffer laid out by attn_block_mask_layout; a caller may also fill the
+ * tables itself (for example per-head block-sparse patterns over MASK_NONE),
+ * as long as every list is ascending and consistent with cls. */
 typedef struct {
+  int Bm, Hm;
   int Sq, Skv, blk_q, blk_kv, n_q_tiles, n_kv_tiles;
-  uint8_t *cls;       /* [n_q_tiles][n_kv_tiles] */
-  int32_t *part_cnt;  /* [n_q_tiles] */
-  int32_t *part_idx;  /* [n_q_tiles][n_kv_tiles], first part_cnt[q] entries valid */
-  int32_t *full_cnt;  /* [n_q_tiles] */
-  int32_t *full_idx;  /* [n_q_tiles][n_kv_tiles], first full_cnt[q] entries valid */
+  uint8_t *cls;       /* [Bm][Hm][n_q_tiles][n_kv_tiles] */
+  int32_t *part_cnt;  /* [Bm][Hm][n_q_tiles] */
+  int32_t *part_idx;  /* [Bm][Hm][n_q_tiles][n_kv_tiles], first part_cnt entries of a row valid */
+  int32_t *full_cnt;  /* [Bm][Hm][n_q_tiles] */
+  int32_t *full_idx;  /* [Bm][Hm][n_q_tiles][n_kv_tiles], first full_cnt entries of a row valid */
+  /* Work order (scheduling only, never changes a result): [Bm][n_q_tiles], the
+   * q-tiles of batch slice b (head slice 0) by decreasing number of visited
+   * kv tiles (part_cnt + full_cnt), ties by index. NULL = last q-tile first.
+   * attn_build_block_mask fills it; a caller filling the tables itself may
+   * set it to NULL or write any permutation. */
+  int32_t *row_order;
+  /* DOCUMENT masks (filled by attn_build_block_mask from the document rows):
+   * doc_sorted[b] = 1 when the ids of row b never decrease, and then
+   * doc_start[b][i] is the first position of the run of equal ids holding i,
+   * so that key j <= i is allowed iff j >= doc_start[b][i] (each document is
+   * one run). Rows with doc_sorted 0 are masked by comparing ids. */
+  int32_t *doc_start; /* [Bm][Sq] */
+  int32_t *doc_sorted;/* [Bm] */
 } attn_block_mask;
 
 /* Bytes of device memory a block mask for these sizes needs (0 if invalid). */
-size_t attn_block_mask_bytes(int Sq, int Skv, int blk_q, int blk_kv);
+size_t attn_block_mask_bytes(int Bm, int Hm, int Sq, int Skv, int blk_q, int blk_kv);
 
 /* Carves the tables out of `buf` (device, >= attn_block_mask_bytes, 16-byte
  * aligned) and fills `out`. Host-only pointer arithmetic; nothing is launched. */
-attn_status attn_block_mask_layout(void *buf, size_t buf_bytes, int Sq, int Skv, int blk_q, int blk_kv,
-                                   attn_block_mask *out);
+attn_status attn_block_mask_layout(void *buf, size_t buf_bytes, int Bm, int Hm, int Sq, int Skv, int blk_q,
+                                   int blk_kv, attn_block_mask *out);
 
 /* Classifies every tile of the mask on the device by evaluating the mask on
  * each in-range (q, kv) pair (out-of-range positions of ragged edge tiles do
- * not count) and writes the class table and both ascending index lists.
- * Any mask kind is accepted; blk_q and blk_kv must be multiples of 16. */
+ * not count) and writes the class tables and both ascending index lists of
+ * every (batch, head) slice. A DOCUMENT mask reads document row b for slice
+ * b (row 0 for every slice when doc_batch_stride is 0); the mask kinds do not
+ * depend on the head, so the Hm slices of a batch are equal. Any mask kind is
+ * accepted; blk_q and blk_kv must be multiples of 16. */
 attn_status attn_build_block_mask(const attn_mask_spec *spec, const attn_block_mask *out, void *stream);
 
 typedef struct {
@@ -119,7 +148,8 @@ typedef struct {
   float scale;                /* softmax_scale; <= 0 selects 1/sqrt(D) */
   attn_mask_spec mask;
   const attn_block_mask *block_mask; /* optional for NONE/CAUSAL/WINDOW, required for
-                                        DOCUMENT; 128 x 128 tiles built for (Sq, Skv) */
+                                        DOCUMENT; 128 x 128 tiles for (Sq, Skv), Bm in {1, B},
+                                        Hm in {1, Hq} */
   attn_mod_kind mod;
   float softcap;              /* SOFTCAP: cap > 0 */
   const float *alibi_slopes;  /* ALIBI: device fp32 [Hq] or [B][Hq] */

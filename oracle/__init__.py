@@ -54,7 +54,7 @@ class _AttnArgs(ctypes.Structure):
         ("scale", ctypes.c_double),
         ("mask", ctypes.c_int), ("window_left", ctypes.c_int), ("window_right", ctypes.c_int),
         ("q_offset", ctypes.c_int),
-        ("doc_id", ctypes.c_void_p),
+        ("doc_id", ctypes.c_void_p), ("doc_bstride", ctypes.c_int64),
         ("mod", ctypes.c_int), ("softcap", ctypes.c_double),
         ("alibi", ctypes.c_void_p), ("alibi_bstride", ctypes.c_int64),
         ("kv_begin", ctypes.c_int), ("kv_end", ctypes.c_int),
@@ -110,7 +110,8 @@ def attn(q, k, v, *, scale: Optional[float] = None, mask: int = MASK_NONE, windo
     """Exact attention forward in fp64.
 
     q: uint16 bf16 bits [B, Sq, Hq, D]; k, v: [B, Skv, Hkv, D] (any strides,
-    last dim contiguous). rows: optional int array [n, 3] of (b, h, i).
+    last dim contiguous). doc_id: [S] (shared by every batch) or [B, S].
+    rows: optional int array [n, 3] of (b, h, i).
     Returns (O, LSE): O float64 [B, Sq, Hq, D] and LSE [B, Hq, Sq] for all rows,
     or O [n, D] and LSE [n] for the given rows.
     """
@@ -129,6 +130,8 @@ def attn(q, k, v, *, scale: Optional[float] = None, mask: int = MASK_NONE, windo
     a.mask, a.window_left, a.window_right, a.q_offset = mask, int(window[0]), int(window[1]), q_offset
     doc = None if doc_id is None else np.ascontiguousarray(doc_id, dtype=np.int32)
     a.doc_id = _ptr(doc)
+    # doc_id [S]: one layout for every batch; [B, S]: row b for batch b
+    a.doc_bstride = doc.shape[1] if doc is not None and doc.ndim == 2 else 0
     a.mod, a.softcap = mod, float(softcap)
     al = None
     if alibi is not None:

@@ -56,7 +56,8 @@ typedef struct {
   int B, Hq, Hkv, Sq, Skv, D;
   double scale;
   int mask, window_left, window_right, q_offset;
-  const int32_t *doc_id;             /* [Sq] == [Skv], document mask only */
+  const int32_t *doc_id;             /* document mask only: row b ([Sq] == [Skv]) at doc_id + b * doc_bstride */
+  int64_t doc_bstride;               /* 0: one row shared by every batch */
   int mod;
   double softcap;
   const float *alibi;                /* alibi[b * alibi_bstride + h] */
@@ -91,10 +92,12 @@ static void attn_row(const oracle_attn_args *a, int b, int h, int i, double *o, 
   const int hk = h / g;
   const int64_t q_pos = (int64_t)i + a->q_offset;
   const uint16_t *qr = a->q + b * a->q_sb + (int64_t)i * a->q_ss + (int64_t)h * a->q_sh;
+  /* the mask_mod sees the batch index: batch b has its own document row */
+  const int32_t *doc = a->doc_id ? a->doc_id + (int64_t)b * a->doc_bstride : NULL;
   double m = -INFINITY;
   int any = 0;
   for (int j = a->kv_begin; j < a->kv_end; ++j) {
-    if (!mask_allows(a->mask, a->window_left, a->window_right, q_pos, j, a->doc_id, i)) {
+    if (!mask_allows(a->mask, a->window_left, a->window_right, q_pos, j, doc, i)) {
       s[j] = -INFINITY;
       continue;
     }

@@ -50,19 +50,27 @@ def test_status_strings(lib):
 
 
 def test_block_mask_sizes_and_layout(lib):
-    n = lib.attn_block_mask_bytes(16384, 16384, 128, 128)
+    n = lib.attn_block_mask_bytes(1, 1, 16384, 16384, 128, 128)
     assert n >= 128 * 128 * (1 + 4 + 4) + 2 * 128 * 4
-    assert lib.attn_block_mask_bytes(0, 10, 128, 128) == 0
+    assert lib.attn_block_mask_bytes(1, 1, 0, 10, 128, 128) == 0
+    assert lib.attn_block_mask_bytes(0, 1, 10, 10, 128, 128) == 0
     bm = _lib.BlockMaskC()
     base = 1 << 20  # host-side arithmetic only: the layout never dereferences
-    assert lib.attn_block_mask_layout(base, n, 16384, 16384, 128, 128, ctypes.byref(bm)) == 0
-    assert (bm.n_q_tiles, bm.n_kv_tiles) == (128, 128)
+    assert lib.attn_block_mask_layout(base, n, 1, 1, 16384, 16384, 128, 128, ctypes.byref(bm)) == 0
+    assert (bm.Bm, bm.Hm, bm.n_q_tiles, bm.n_kv_tiles) == (1, 1, 128, 128)
     ptrs = [bm.cls, bm.part_cnt, bm.full_cnt, bm.part_idx, bm.full_idx]
     assert all(p % 16 == 0 for p in ptrs) and ptrs == sorted(ptrs)
     assert bm.full_idx + 128 * 128 * 4 <= base + n
-    assert lib.attn_block_mask_layout(base, n - 1, 16384, 16384, 128, 128, ctypes.byref(bm)) == _lib.ATTN_ERR_WORKSPACE
-    assert lib.attn_block_mask_layout(base + 4, n, 16384, 16384, 128, 128, ctypes.byref(bm)) == \
+    assert lib.attn_block_mask_layout(base, n - 1, 1, 1, 16384, 16384, 128, 128, ctypes.byref(bm)) == \
+        _lib.ATTN_ERR_WORKSPACE
+    assert lib.attn_block_mask_layout(base + 4, n, 1, 1, 16384, 16384, 128, 128, ctypes.byref(bm)) == \
         _lib.ATTN_ERR_INVALID_ARG
+    # per-batch and per-head slices: every table scales with Bm * Hm
+    n6 = lib.attn_block_mask_bytes(2, 3, 1000, 700, 128, 128)
+    assert lib.attn_block_mask_layout(base, n6, 2, 3, 1000, 700, 128, 128, ctypes.byref(bm)) == 0
+    nq, nk = 8, 6
+    assert bm.part_cnt - bm.cls >= 6 * nq * nk and bm.full_cnt - bm.part_cnt >= 6 * nq * 4
+    assert bm.full_idx - bm.part_idx >= 6 * nq * nk * 4 and bm.full_idx + 6 * nq * nk * 4 <= base + n6
 
 
 def test_decode_workspace_bytes(lib):
@@ -112,6 +120,20 @@ def test_fwd_bad_strides_and_document_mask(lib):
     p = _fwd_params()
     p.mask.kind = _lib.MASK_DOCUMENT  # no doc ids, no block mask
     assert lib.attn_fwd(ctypes.byref(p), None) == _lib.ATTN_ERR_INVALID_ARG
+    # a block mask whose batch / head slices match neither 1 nor the call's B / Hq
+    bm = _lib.BlockMaskC()
+    nb = lib.attn_block_mask_bytes(3, 1, 128, 128, 128, 128)
+    assert lib.attn_block_mask_layout(1 << 20, nb, 3, 1, 128, 128, 128, 128, ctypes.byref(bm)) == 0
+    p = _fwd_params()
+    p.block_mask = ctypes.pointer(bm)
+    assert lib.attn_fwd(ctypes.byref(p), None) == _lib.ATTN_ERR_INVALID_ARG
+    # document rows must be 16-byte strided
+    p = _fwd_params()
+    p.mask.kind, p.mask.doc_id, p.mask.doc_batch_stride = _lib.MASK_DOCUMENT, 1 << 20, 130
+    nb = lib.attn_block_mask_bytes(1, 1, 128, 128, 128, 128)
+    assert lib.attn_block_mask_layout(1 << 20, nb, 1, 1, 128, 128, 128, 128, ctypes.byref(bm)) == 0
+    p.block_mask = ctypes.pointer(bm)
+    assert lib.attn_fwd(ctypes.byref(p), None) == _lib.ATTN_ERR_UNSUPPORTED
     assert lib.attn_fwd(None, None) == _lib.ATTN_ERR_INVALID_ARG
     assert lib.attn_fwd(ctypes.byref(_fwd_params(B=0)), None) == _lib.ATTN_OK  # empty batch: nothing to do
 

@@ -150,12 +150,13 @@ def test_explicit_scale():
 
 # ------------------------------------------------------------ block mask builder (exact)
 
-def _bm_compare(bm, ref):
-    cls = bm.cls.cpu().numpy()
+def _bm_compare(bm, ref, b=0, h=0):
+    """Slice (b, h) of a device block mask against the oracle's tables."""
+    cls = bm.cls.cpu().numpy()[b, h]
     assert np.array_equal(cls, ref["cls"])
-    pc, fc = bm.part_cnt.cpu().numpy(), bm.full_cnt.cpu().numpy()
+    pc, fc = bm.part_cnt.cpu().numpy()[b, h], bm.full_cnt.cpu().numpy()[b, h]
     assert np.array_equal(pc, ref["part_cnt"]) and np.array_equal(fc, ref["full_cnt"])
-    pi, fi = bm.part_idx.cpu().numpy(), bm.full_idx.cpu().numpy()
+    pi, fi = bm.part_idx.cpu().numpy()[b, h], bm.full_idx.cpu().numpy()[b, h]
     for r in range(cls.shape[0]):
         assert np.array_equal(pi[r, :pc[r]], ref["part_idx"][r, :pc[r]])
         assert np.array_equal(fi[r, :fc[r]], ref["full_idx"][r, :fc[r]])
@@ -216,6 +217,136 @@ def test_block_mask_window_edges_exact(window, q_off):
         bm = ea.attn_build_block_mask(Sq, Skv, window=window, q_offset=q_off, blk_q=blk, blk_kv=blk)
         torch.cuda.synchronize()
         _bm_compare(bm, ref)
+
+
+def test_block_mask_per_batch_documents_and_head_slices_exact():
+    """Bm = 2 batches with different document layouts, Hm = 3 head slices: each
+    slice equals the oracle's tables for its batch's document row."""
+    S = 1500
+    doc = np.stack([W.doc_ids_from_lengths(W.doc_lengths(7, S, 60, 500)),
+                    W.doc_ids_from_lengths(W.doc_lengths(8, S, 200, 900))])
+    bm = ea.attn_build_block_mask(S, S, doc_id=torch.from_numpy(doc).cuda(), H=3)
+    torch.cuda.synchronize()
+    assert bm.shape[:2] == (2, 3)
+    for b in range(2):
+        ref = oracle.block_mask(W.MASK_DOCUMENT, S, S, doc_id=doc[b])
+        for h in range(3):
+            _bm_compare(bm, ref, b, h)
+    # window mask with head slices (no batch dependence): every slice equal
+    bm = ea.attn_build_block_mask(1000, 1000, window=(300, 0), B=2, H=2)
+    torch.cuda.synchronize()
+    ref = oracle.block_mask(W.MASK_WINDOW, 1000, 1000, window=(300, 0))
+    for b in range(2):
+        for h in range(2):
+            _bm_compare(bm, ref, b, h)
+
+
+def _runs_and_order(doc_row, ref):
+    """Document run starts, the never-decreasing flag and the heaviest-first
+    q-tile order, from their definitions (host reference for the builder)."""
+    S = len(doc_row)
+    start = np.zeros(S, np.int32)
+    for i in range(1, S):
+        start[i] = start[i - 1] if doc_row[i] == doc_row[i - 1] else i
+    sorted_ = int(np.all(np.diff(doc_row) >= 0))
+    wgt = ref["part_cnt"] + ref["full_cnt"]
+    order = np.array(sorted(range(len(wgt)), key=lambda i: (-wgt[i], i)), np.int32)
+    return start, sorted_, order
+
+
+@pytest.mark.parametrize("ids", ["sorted", "unsorted"])
+def test_block_mask_document_runs_and_work_order_exact(ids):
+    S = 3001
+    if ids == "sorted":
+        doc = np.stack([W.doc_ids_from_lengths(W.doc_lengths(27, S, 100, 900)),
+                        W.doc_ids_from_lengths(W.doc_lengths(28, S, 30, 200))])
+    else:
+        doc = np.stack([W.uniform_ints(29, S, 0, 3), W.doc_ids_from_lengths(W.doc_lengths(30, S, 30, 200))])
+    bm = ea.attn_build_block_mask(S, S, doc_id=torch.from_numpy(doc).cuda())
+    torch.cuda.synchronize()
+    for b in range(2):
+        ref = oracle.block_mask(W.MASK_DOCUMENT, S, S, doc_id=doc[b])
+        start, sorted_, order = _runs_and_order(doc[b], ref)
+        assert np.array_equal(bm.doc_start.cpu().numpy()[b], start)
+        assert int(bm.doc_sorted.cpu().numpy()[b]) == sorted_
+        assert np.array_equal(bm.row_order.cpu().numpy()[b], order)
+    assert int(bm.doc_sorted.cpu().numpy()[0]) == (1 if ids == "sorted" else 0)
+
+
+@pytest.mark.parametrize("S", [777, 1030])
+def test_documents_unsorted_ids_forward(S):
+    """Ids that go up and down (every position compared by id, the path for
+    documents that are not one run each), ragged lengths included."""
+    doc = W.uniform_ints(31 + S, S, 0, 2)
+    full_case(1, S, 4, 2, 128, seed=87 + S, doc_id_np=doc)
+    full_case(1, S, 2, 2, 64, seed=88 + S, doc_id_np=doc, alibi_np=W.alibi_slopes(2))
+
+
+def test_per_batch_documents_forward():
+    """B = 2 packed-document batches with different layouts through attn_fwd
+    (doc_id [B, S], block mask with Bm = 2), GQA and ALiBi, against the oracle."""
+    S = 1300
+    doc = np.stack([W.doc_ids_from_lengths(W.doc_lengths(17, S, 128, 700)),
+                    W.doc_ids_from_lengths(W.doc_lengths(18, S, 40, 300))])
+    full_case(2, S, 8, 2, 128, seed=88, doc_id_np=doc, alibi_np=W.alibi_slopes(8))
+    full_case(2, S, 3, 3, 64, seed=89, doc_id_np=doc)
+
+
+def test_per_head_block_sparse_tables_filled_by_the_caller():
+    """A caller-filled block mask with Hm = Hq over MASK_NONE: heads 0 and 2
+    attend block-causally (every key of tiles up to the query's own tile),
+    heads 1 and 3 to every key. The oracle computes each row over its allowed
+    key range (kv_range), the plain definition on a key subset."""
+    B, S, Hq, Hkv, D = 1, 700, 4, 2, 128
+    nT = -(-S // 128)
+    cls = np.zeros((1, Hq, nT, nT), np.uint8)
+    for h in range(Hq):
+        for i in range(nT):
+            for j in range(nT):
+                full = j < nT - 1 or S % 128 == 0
+                allowed = (j <= i) if h % 2 == 0 else True
+                cls[0, h, i, j] = 0 if not allowed else (2 if full else 1)
+    bm = ea.BlockMask(S, S, 128, 128, torch.device("cuda"), Bm=1, Hm=Hq)
+    bm.cls.copy_(torch.from_numpy(cls))
+    pc = (cls == 1).sum(-1).astype(np.int32)
+    fc = (cls == 2).sum(-1).astype(np.int32)
+    pi = np.zeros(cls.shape, np.int32)
+    fi = np.zeros(cls.shape, np.int32)
+    for h in range(Hq):
+        for i in range(nT):
+            p_, f_ = np.nonzero(cls[0, h, i] == 1)[0], np.nonzero(cls[0, h, i] == 2)[0]
+            pi[0, h, i, :len(p_)] = p_
+            fi[0, h, i, :len(f_)] = f_
+    for name, arr in (("part_cnt", pc), ("full_cnt", fc), ("part_idx", pi), ("full_idx", fi)):
+        getattr(bm, name).copy_(torch.from_numpy(arr))
+    q = W.normal_bf16(91, (B, S, Hq, D))
+    k = W.normal_bf16(92, (B, S, Hkv, D))
+    v = W.normal_bf16(93, (B, S, Hkv, D))
+    o_plain, l_plain = oracle.attn(q, k, v)
+    ref_o = np.empty((S, Hq, D))
+    ref_l = np.empty((Hq, S))
+    for h in range(Hq):
+        for i in range(S):
+            if h % 2 == 1:
+                ref_o[i, h], ref_l[h, i] = o_plain[0, i, h], l_plain[0, h, i]
+            else:
+                ro, rl = oracle.attn(q, k, v, rows=np.array([[0, h, i]]), kv_range=(0, min(S, (i // 128 + 1) * 128)))
+                ref_o[i, h], ref_l[h, i] = ro[0], rl[0]
+    # no work order (NULL), then an explicit permutation of the q-tiles
+    bm.c.row_order = None
+    o, lse = run_fwd(q, k, v, block_mask=bm)
+    compare(o[0], ref_o, lse[0], ref_l, "per-head tables, no order")
+    bm2 = ea.attn_build_block_mask(S, S, device=torch.device("cuda"))  # only its order table is used
+    bm.c.row_order = bm2.c.row_order
+    bm2.row_order.copy_(torch.tensor([[3, 0, 5, 1, 4, 2]], dtype=torch.int32))
+    o, lse = run_fwd(q, k, v, block_mask=bm)
+    compare(o[0], ref_o, lse[0], ref_l, "per-head tables, permuted order")
+    # an order entry outside the q-tiles is reported and not followed
+    bm2.row_order.copy_(torch.tensor([[3, 0, 99, 1, 4, 2]], dtype=torch.int32))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o3, _ = ea.attn_fwd(dev_bf16(q), dev_bf16(k), dev_bf16(v), block_mask=bm, status=status)
+    torch.cuda.synchronize()
+    assert status.item() & ea.ATTN_DEV_BAD_MASK
 
 
 def test_block_mask_drives_causal_like_analytic():

@@ -61,3 +61,37 @@ def test_bench_flop_accounting_matches_the_oracle_pair_count(name):
         kw = dict(doc_id=W.doc_ids_from_lengths(doc_lens))
     per_head = oracle.count_pairs(w.mask, S, S, **kw)
     assert bench.unmasked_pairs(ws, doc_lens) == per_head * w.B * w.Hq
+
+
+def test_trace_summary_on_synthetic_records():
+    """The cycle-trace summarizer (trace build analysis) on a hand-made record
+    stream: one CTA, two units of 2 and 1 steps on subtile 0."""
+    import numpy as np
+    from exact_attention_145_b200 import trace as T
+    E = T.EV
+    per = 64
+    raw = np.zeros((1, T.N_ROLES, per, 2), np.uint32)
+
+    def put(role, recs):
+        for i, (t, e, aux) in enumerate(recs):
+            raw[0, role, i] = (t, (e << 24) | aux)
+
+    put(0, [(10, E["S_WAIT"], 0), (100, E["S_READY"], 0 | (2 << 20)), (1100, E["P_DONE"], 0),
+            (1110, E["S_WAIT"], 1), (2000, E["S_READY"], 1 | (1 << 20)), (3500, E["P_DONE"], 1),
+            (3510, E["O_WAIT"], 0), (3800, E["EPI_BEGIN"], 0), (4400, E["EPI_END"], 0),
+            (4410, E["S_WAIT"], 2), (6000, E["S_READY"], 2 | (2 << 20)), (7000, E["P_DONE"], 2),
+            (7010, E["O_WAIT"], 1), (7300, E["EPI_BEGIN"], 1), (7900, E["EPI_END"], 1),
+            (8000, E["KERNEL_END"], 0)])
+    put(T.MMA, [(900, E["P_WAIT"], 0), (1150, E["PV"], 0)])
+    # warps 1-3 of subtile 0 hand over P of step 0 later than warp 0
+    for w, late in ((1, 40), (2, 300), (3, 10)):
+        put(w, [(1100 + late, E["P_DONE"], 0)])
+    s = T.summarize(T.decode_records(raw, 1, per))
+    assert s["prologue_to_first_s"] == 100
+    assert s["softmax_full_tile"] == 1000 and s["softmax_partial_tile"] == 1500
+    assert s["p_to_next_s"] == 900 and s["step_period_per_subtile"] == 1900
+    assert s["unit_boundary"] == 6000 - 3500
+    assert s["epilogue"] == 600 and s["o_wait_before_epilogue"] == 290
+    assert s["mma_wait_for_p"] == 250
+    assert s["p_handover_skew_across_warps"] == 300
+    assert s["critical_cta"] == {"cycles": 8000, "steps": 3, "units": 2}

@@ -92,6 +92,31 @@ def test_uniform_scores_average_allowed_values(mask, window):
         assert np.max(np.abs(o[0, i] - want)) < 1e-14
 
 
+def test_uniform_scores_per_batch_documents():
+    # FlexAttention's mask_mod receives the batch index (attention-gym issue 101:
+    # create_block_mask(mask_mod, B, H, Q_LEN, KV_LEN)), so a batch of packed
+    # sequences may have a different document layout per batch. With q = 0 the
+    # row of batch b averages the V rows of its own document up to i; the
+    # document start comes from that batch's lengths by interval arithmetic.
+    S, H, D = 23, 2, 4
+    q = np.zeros((2, S, H, D), np.uint16)
+    _, k, v = rand_qkv(12, 2, S, H, H, D)
+    lens = [[5, 1, 9, 8], [11, 12]]
+    doc = np.stack([W.doc_ids_from_lengths(x) for x in lens])
+    o, lse = oracle.attn(q, k, v, mask=W.MASK_DOCUMENT, doc_id=doc)
+    vf = f64(v)
+    for b in range(2):
+        starts = np.concatenate([[0], np.cumsum(lens[b])[:-1]])
+        for i in range(S):
+            lo = starts[doc[b, i]]
+            assert abs(lse[b, 1, i] - math.log(i - lo + 1)) < 1e-14
+            assert np.max(np.abs(o[b, i] - vf[b, lo:i + 1].mean(axis=0))) < 1e-14
+    # a [S] row is shared by every batch: equal to passing it once per batch
+    o1, l1 = oracle.attn(q, k, v, mask=W.MASK_DOCUMENT, doc_id=doc[0])
+    o2, l2 = oracle.attn(q, k, v, mask=W.MASK_DOCUMENT, doc_id=np.stack([doc[0], doc[0]]))
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
 def test_constant_v_rows_give_that_row():
     q, k, _ = rand_qkv(21, 2, 37, 4, 2, 16)
     row = W.normal_bf16(99, (16,))
