@@ -74,6 +74,23 @@ class _DecodeArgs(ctypes.Structure):
     ]
 
 
+class _F64Args(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("dout", ctypes.c_void_p),
+        ("q_sb", ctypes.c_int64), ("q_ss", ctypes.c_int64), ("q_sh", ctypes.c_int64),
+        ("k_sb", ctypes.c_int64), ("k_ss", ctypes.c_int64), ("k_sh", ctypes.c_int64),
+        ("v_sb", ctypes.c_int64), ("v_ss", ctypes.c_int64), ("v_sh", ctypes.c_int64),
+        ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+        ("Sq", ctypes.c_int), ("Skv", ctypes.c_int), ("D", ctypes.c_int),
+        ("scale", ctypes.c_double),
+        ("mask", ctypes.c_int), ("window_left", ctypes.c_int), ("window_right", ctypes.c_int),
+        ("q_offset", ctypes.c_int),
+        ("doc_id", ctypes.c_void_p), ("doc_bstride", ctypes.c_int64),
+        ("mod", ctypes.c_int), ("softcap", ctypes.c_double),
+        ("alibi", ctypes.c_void_p), ("alibi_bstride", ctypes.c_int64),
+    ]
+
+
 def _load():
     global _lib
     with _lock:
@@ -92,6 +109,11 @@ def _load():
             lib.oracle_block_mask.restype = ctypes.c_int
             lib.oracle_count_pairs.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] + [ctypes.c_int] * 2
             lib.oracle_count_pairs.restype = ctypes.c_int64
+            lib.oracle_attn_f64.argtypes = [ctypes.POINTER(_F64Args), ctypes.c_void_p, ctypes.c_void_p]
+            lib.oracle_attn_f64.restype = ctypes.c_int
+            lib.oracle_attn_bwd_f64.argtypes = [ctypes.POINTER(_F64Args), ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_int]
+            lib.oracle_attn_bwd_f64.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -235,3 +257,68 @@ def count_pairs(mask: int, Sq: int, Skv: int, window=(-1, -1), q_offset: int = 0
     lib = _load()
     doc = None if doc_id is None else np.ascontiguousarray(doc_id, dtype=np.int32)
     return int(lib.oracle_count_pairs(mask, int(window[0]), int(window[1]), q_offset, _ptr(doc), Sq, Skv))
+
+
+def _f64_args(q, k, v, dout, scale, mask, window, q_offset, doc_id, mod, softcap, alibi, keep):
+    for t in (q, k, v) + (() if dout is None else (dout,)):
+        assert t.dtype == np.float64 and t.ndim == 4 and t.strides[3] == 8
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    a = _F64Args()
+    a.q, a.k, a.v = q.ctypes.data, k.ctypes.data, v.ctypes.data
+    a.dout = None if dout is None else dout.ctypes.data
+    if dout is not None:
+        assert dout.shape == q.shape and dout.strides == q.strides
+    a.q_sb, a.q_ss, a.q_sh = (x // 8 for x in q.strides[:3])
+    a.k_sb, a.k_ss, a.k_sh = (x // 8 for x in k.strides[:3])
+    a.v_sb, a.v_ss, a.v_sh = (x // 8 for x in v.strides[:3])
+    a.B, a.Hq, a.Hkv, a.Sq, a.Skv, a.D = B, Hq, Hkv, Sq, Skv, D
+    a.scale = (1.0 / np.sqrt(D)) if scale is None else float(scale)
+    a.mask, a.window_left, a.window_right, a.q_offset = mask, int(window[0]), int(window[1]), q_offset
+    doc = None if doc_id is None else np.ascontiguousarray(doc_id, dtype=np.int32)
+    a.doc_id = _ptr(doc)
+    a.doc_bstride = doc.shape[1] if doc is not None and doc.ndim == 2 else 0
+    a.mod, a.softcap = mod, float(softcap)
+    al = None
+    if alibi is not None:
+        al = np.ascontiguousarray(alibi, dtype=np.float32)
+        a.alibi_bstride = Hq if al.ndim == 2 else 0
+    a.alibi = _ptr(al)
+    keep.extend([doc, al])
+    return a
+
+
+def attn_f64(q, k, v, *, scale: Optional[float] = None, mask: int = MASK_NONE, window=(-1, -1),
+             q_offset: int = 0, doc_id=None, mod: int = MOD_NONE, softcap: float = 0.0, alibi=None):
+    """The forward on float64 inputs [B, S, H, D] (no bf16 rounding), for
+    finite-difference checks of the backward. Returns (O [B, Sq, Hq, D], LSE [B, Hq, Sq])."""
+    lib = _load()
+    keep = []
+    a = _f64_args(q, k, v, None, scale, mask, window, q_offset, doc_id, mod, softcap, alibi, keep)
+    B, Sq, Hq, D = q.shape
+    o = np.empty((B, Sq, Hq, D), dtype=np.float64)
+    lse = np.empty((B, Hq, Sq), dtype=np.float64)
+    if lib.oracle_attn_f64(ctypes.byref(a), o.ctypes.data, lse.ctypes.data) != 0:
+        raise ValueError("oracle_attn_f64: bad arguments")
+    return o, lse
+
+
+def attn_bwd(q, k, v, dout, *, scale: Optional[float] = None, mask: int = MASK_NONE, window=(-1, -1),
+             q_offset: int = 0, doc_id=None, mod: int = MOD_NONE, softcap: float = 0.0, alibi=None,
+             nthreads: Optional[int] = None):
+    """Gradients of the attention forward with respect to q, k, v for the
+    upstream gradient dout = dL/dO, by the chain rule in fp64. Inputs are
+    float64 [B, S, H, D] (widen bf16 bits with workloads.bf16_bits_to_f64).
+    Returns (dq [B, Sq, Hq, D], dk [B, Skv, Hkv, D], dv [B, Skv, Hkv, D])."""
+    lib = _load()
+    keep = []
+    a = _f64_args(q, k, v, dout, scale, mask, window, q_offset, doc_id, mod, softcap, alibi, keep)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    dq = np.empty((B, Sq, Hq, D), dtype=np.float64)
+    dk = np.empty((B, Skv, Hkv, D), dtype=np.float64)
+    dv = np.empty((B, Skv, Hkv, D), dtype=np.float64)
+    nt = default_threads() if nthreads is None else nthreads
+    if lib.oracle_attn_bwd_f64(ctypes.byref(a), dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, nt) != 0:
+        raise ValueError("oracle_attn_bwd_f64: bad arguments")
+    return dq, dk, dv

@@ -354,3 +354,184 @@ int64_t oracle_count_pairs(int mask, int window_left, int window_right, int q_of
     for (int j = 0; j < Skv; ++j) n += mask_allows(mask, window_left, window_right, (int64_t)i + q_offset, j, doc_id, i);
   return n;
 }
+
+/* ------------------------------------------------------------ fp64-input forward and backward */
+
+/* The same attention in double precision on double inputs (no bf16 step):
+ * the forward exists so that the backward can be checked against central
+ * finite differences of it. Layouts as in oracle_attn_args (element strides
+ * of batch, sequence, head; last dimension contiguous). */
+typedef struct {
+  const double *q, *k, *v, *dout;    /* dout: upstream gradient dL/dO, laid out like q */
+  int64_t q_sb, q_ss, q_sh;
+  int64_t k_sb, k_ss, k_sh;
+  int64_t v_sb, v_ss, v_sh;
+  int B, Hq, Hkv, Sq, Skv, D;
+  double scale;
+  int mask, window_left, window_right, q_offset;
+  const int32_t *doc_id;
+  int64_t doc_bstride;
+  int mod;
+  double softcap;
+  const float *alibi;
+  int64_t alibi_bstride;
+} oracle_f64_args;
+
+static double f64_score(const oracle_f64_args *a, int b, int h, int i, int j, double *dmod) {
+  /* z = scale * q.k; s = mod(z); *dmod = ds/dz */
+  const int g = a->Hq / a->Hkv, hk = h / g;
+  const double *qr = a->q + b * a->q_sb + (int64_t)i * a->q_ss + (int64_t)h * a->q_sh;
+  const double *kr = a->k + b * a->k_sb + (int64_t)j * a->k_ss + (int64_t)hk * a->k_sh;
+  double dot = 0.0;
+  for (int d = 0; d < a->D; ++d) dot += qr[d] * kr[d];
+  const double z = a->scale * dot;
+  if (a->mod == O_MOD_SOFTCAP) {
+    const double t = tanh(z / a->softcap);
+    *dmod = 1.0 - t * t;
+    return a->softcap * t;
+  }
+  *dmod = 1.0;
+  if (a->mod == O_MOD_ALIBI) {
+    const int64_t q_pos = (int64_t)i + a->q_offset;
+    return z + (double)a->alibi[b * a->alibi_bstride + h] * (double)(j - q_pos);
+  }
+  return z;
+}
+
+static int f64_allowed(const oracle_f64_args *a, int b, int i, int j) {
+  const int32_t *doc = a->doc_id ? a->doc_id + (int64_t)b * a->doc_bstride : NULL;
+  return mask_allows(a->mask, a->window_left, a->window_right, (int64_t)i + a->q_offset, j, doc, i);
+}
+
+/* Row (b, h, i): p[j] = softmax probabilities (0 where masked), returns LSE
+ * (-inf for a row with no allowed key, then p = 0). */
+static double f64_row_probs(const oracle_f64_args *a, int b, int h, int i, double *p, double *dm) {
+  double m = -INFINITY;
+  for (int j = 0; j < a->Skv; ++j) {
+    if (!f64_allowed(a, b, i, j)) {
+      p[j] = -INFINITY;
+      continue;
+    }
+    p[j] = f64_score(a, b, h, i, j, &dm[j]);
+    if (p[j] > m) m = p[j];
+  }
+  if (m == -INFINITY) {
+    for (int j = 0; j < a->Skv; ++j) p[j] = 0.0;
+    return -INFINITY;
+  }
+  double l = 0.0;
+  for (int j = 0; j < a->Skv; ++j) {
+    p[j] = p[j] == -INFINITY ? 0.0 : exp(p[j] - m);
+    l += p[j];
+  }
+  for (int j = 0; j < a->Skv; ++j) p[j] /= l;
+  return m + log(l);
+}
+
+/* o: [B][Sq][Hq][D] contiguous, lse: [B][Hq][Sq]. Returns 0 or -1. */
+int oracle_attn_f64(const oracle_f64_args *a, double *o, double *lse) {
+  if (a->Hkv <= 0 || a->Hq % a->Hkv != 0 || a->D <= 0) return -1;
+  double *p = (double *)malloc(sizeof(double) * (size_t)(a->Skv > 0 ? a->Skv : 1));
+  double *dm = (double *)malloc(sizeof(double) * (size_t)(a->Skv > 0 ? a->Skv : 1));
+  const int g = a->Hq / a->Hkv;
+  for (int b = 0; b < a->B; ++b)
+    for (int h = 0; h < a->Hq; ++h)
+      for (int i = 0; i < a->Sq; ++i) {
+        const double L = f64_row_probs(a, b, h, i, p, dm);
+        lse[((int64_t)b * a->Hq + h) * a->Sq + i] = L;
+        double *orow = o + (((int64_t)b * a->Sq + i) * a->Hq + h) * a->D;
+        for (int d = 0; d < a->D; ++d) orow[d] = 0.0;
+        for (int j = 0; j < a->Skv; ++j) {
+          if (p[j] == 0.0) continue;
+          const double *vr = a->v + b * a->v_sb + (int64_t)j * a->v_ss + (int64_t)(h / g) * a->v_sh;
+          for (int d = 0; d < a->D; ++d) orow[d] += p[j] * vr[d];
+        }
+      }
+  free(p);
+  free(dm);
+  return 0;
+}
+
+/* Backward of the forward above by the chain rule (FlashAttention overview,
+ * "Examples": the backward pass and its deterministic option): with
+ * p = softmax row, dp_ij = dO_i . v_j, ds_ij = p_ij (dp_ij - sum_j' p_ij' dp_ij'),
+ * dz_ij = ds_ij * mod'(z_ij),
+ *   dV_j += p_ij dO_i,  dQ_i = scale sum_j dz_ij k_j,  dK_j += scale dz_ij q_i,
+ * summed over every query head of a KV head's group (GQA) and every row.
+ * One thread per (batch, KV head) owns that head's dK / dV rows.
+ * dq: [B][Sq][Hq][D], dk / dv: [B][Skv][Hkv][D], all contiguous. */
+typedef struct {
+  const oracle_f64_args *a;
+  int bh0, bh1;
+  double *dq, *dk, *dv;
+} bwd_job;
+
+static void *bwd_worker(void *ptr) {
+  bwd_job *job = (bwd_job *)ptr;
+  const oracle_f64_args *a = job->a;
+  const int g = a->Hq / a->Hkv;
+  const size_t n = (size_t)(a->Skv > 0 ? a->Skv : 1);
+  double *p = (double *)malloc(sizeof(double) * n);
+  double *dm = (double *)malloc(sizeof(double) * n);
+  double *dp = (double *)malloc(sizeof(double) * n);
+  for (int bh = job->bh0; bh < job->bh1; ++bh) {
+    const int b = bh / a->Hkv, hk = bh % a->Hkv;
+    for (int h = hk * g; h < hk * g + g; ++h)
+      for (int i = 0; i < a->Sq; ++i) {
+        const double L = f64_row_probs(a, b, h, i, p, dm);
+        double *dqr = job->dq + (((int64_t)b * a->Sq + i) * a->Hq + h) * a->D;
+        for (int d = 0; d < a->D; ++d) dqr[d] = 0.0;
+        if (L == -INFINITY) continue;
+        const double *dor = a->dout + b * a->q_sb + (int64_t)i * a->q_ss + (int64_t)h * a->q_sh;
+        const double *qr = a->q + b * a->q_sb + (int64_t)i * a->q_ss + (int64_t)h * a->q_sh;
+        double Di = 0.0;
+        for (int j = 0; j < a->Skv; ++j) {
+          dp[j] = 0.0;
+          if (p[j] == 0.0) continue;
+          const double *vr = a->v + b * a->v_sb + (int64_t)j * a->v_ss + (int64_t)hk * a->v_sh;
+          for (int d = 0; d < a->D; ++d) dp[j] += dor[d] * vr[d];
+          Di += p[j] * dp[j];
+        }
+        for (int j = 0; j < a->Skv; ++j) {
+          if (p[j] == 0.0) continue;
+          const double dz = p[j] * (dp[j] - Di) * dm[j];
+          const double *kr = a->k + b * a->k_sb + (int64_t)j * a->k_ss + (int64_t)hk * a->k_sh;
+          double *dkr = job->dk + (((int64_t)b * a->Skv + j) * a->Hkv + hk) * a->D;
+          double *dvr = job->dv + (((int64_t)b * a->Skv + j) * a->Hkv + hk) * a->D;
+          for (int d = 0; d < a->D; ++d) {
+            dqr[d] += a->scale * dz * kr[d];
+            dkr[d] += a->scale * dz * qr[d];
+            dvr[d] += p[j] * dor[d];
+          }
+        }
+      }
+  }
+  free(p);
+  free(dm);
+  free(dp);
+  return NULL;
+}
+
+int oracle_attn_bwd_f64(const oracle_f64_args *a, double *dq, double *dk, double *dv, int nthreads) {
+  if (a->Hkv <= 0 || a->Hq % a->Hkv != 0 || a->D <= 0 || a->dout == NULL) return -1;
+  if (a->mask == O_MASK_DOCUMENT && (a->doc_id == NULL || a->Sq != a->Skv || a->q_offset != 0)) return -1;
+  if (a->mod == O_MOD_ALIBI && a->alibi == NULL) return -1;
+  if (a->mod == O_MOD_SOFTCAP && !(a->softcap > 0.0)) return -1;
+  const size_t nkv = (size_t)a->B * a->Skv * a->Hkv * a->D;
+  for (size_t x = 0; x < nkv; ++x) dk[x] = dv[x] = 0.0;
+  const int nbh = a->B * a->Hkv;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > nbh) nthreads = nbh > 0 ? nbh : 1;
+  bwd_job *jobs = (bwd_job *)malloc(sizeof(bwd_job) * (size_t)nthreads);
+  for (int t = 0; t < nthreads; ++t) {
+    jobs[t].a = a;
+    jobs[t].bh0 = nbh * t / nthreads;
+    jobs[t].bh1 = nbh * (t + 1) / nthreads;
+    jobs[t].dq = dq;
+    jobs[t].dk = dk;
+    jobs[t].dv = dv;
+  }
+  run_jobs(bwd_worker, jobs, sizeof(bwd_job), nthreads);
+  free(jobs);
+  return 0;
+}
