@@ -27,7 +27,8 @@ MOD_NONE, MOD_SOFTCAP, MOD_ALIBI = range(3)
 
 EXPORTS = ("attn_block_mask_bytes", "attn_block_mask_layout", "attn_build_block_mask", "attn_fwd",
            "attn_decode_num_splits", "attn_decode_workspace_bytes", "attn_decode", "attn_lse_combine",
-           "attn_status_str", "attn_decode_noalloc", "attn_selftest_wait_timeout")
+           "attn_status_str", "attn_decode_noalloc", "attn_selftest_wait_timeout", "attn_bwd_workspace_bytes",
+           "attn_bwd")
 ATTN_DECODE_NOALLOC_MAX_BYTES = 32 * 1024 * 1024
 
 c_i64x3 = ctypes.c_int64 * 3
@@ -57,6 +58,17 @@ class FwdParams(ctypes.Structure):
                 ("mask", MaskSpec), ("block_mask", ctypes.POINTER(BlockMaskC)),
                 ("mod", ctypes.c_int), ("softcap", ctypes.c_float), ("alibi_slopes", ctypes.c_void_p),
                 ("alibi_batch_stride", ctypes.c_int), ("status", ctypes.c_void_p)]
+
+
+class BwdParams(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("o", ctypes.c_void_p),
+                ("dout", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p),
+                ("q_stride", c_i64x3), ("k_stride", c_i64x3), ("v_stride", c_i64x3), ("o_stride", c_i64x3),
+                ("do_stride", c_i64x3), ("dq_stride", c_i64x3), ("dk_stride", c_i64x3), ("dv_stride", c_i64x3),
+                ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("Sq", ctypes.c_int),
+                ("Skv", ctypes.c_int), ("D", ctypes.c_int), ("scale", ctypes.c_float),
+                ("mask", MaskSpec), ("deterministic", ctypes.c_int), ("status", ctypes.c_void_p)]
 
 
 class DecodeParams(ctypes.Structure):
@@ -106,6 +118,10 @@ def load() -> ctypes.CDLL:
         lib.attn_decode.restype = ctypes.c_int
         lib.attn_decode_noalloc.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_void_p]
         lib.attn_decode_noalloc.restype = ctypes.c_int
+        lib.attn_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 3
+        lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.attn_bwd.argtypes = [ctypes.POINTER(BwdParams), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+        lib.attn_bwd.restype = ctypes.c_int
         lib.attn_lse_combine.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_lse_combine.restype = ctypes.c_int

@@ -12,6 +12,7 @@
 
 #include "../../include/attn.h"
 #include "aux_kernels.cuh"
+#include "bwd_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 using namespace attn_kernels;
@@ -170,9 +171,142 @@ attn_status check_mods(attn_mod_kind mod, float softcap, const float* alibi, int
   return ATTN_OK;
 }
 
+// Backward launches: the smem opt-in is per device and kernel.
+template <typename K>
+attn_status opt_in_smem(K kernel, int bytes, uint64_t& ready_mask, std::mutex& mu) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!(ready_mask & (1ull << dev))) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    ready_mask |= 1ull << dev;
+  }
+  return ATTN_OK;
+}
+
+template <int D>
+attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                       attn_bwd_kernels::BwdArgs a, cudaStream_t st) {
+  using namespace attn_bwd_kernels;
+  using L = BLayout<D>;
+  static std::mutex mu1, mu2;
+  static uint64_t r1 = 0, r2 = 0;
+  if (attn_status e = opt_in_smem(attn_bwd_dkdv_kernel<D>, L::kSmemBytes, r1, mu1)) return e;
+  if (attn_status e = opt_in_smem(attn_bwd_dq_kernel<D>, L::kSmemBytes, r2, mu2)) return e;
+  const int sms = sm_count();
+  a.n_units = a.B * a.Hkv * a.nK;
+  if (a.n_units > 0)
+    attn_bwd_dkdv_kernel<D><<<a.n_units < sms ? a.n_units : sms, kBwdThreads, L::kSmemBytes, st>>>(mq, mk, mv, mdo,
+                                                                                                    a);
+  a.n_units = a.B * a.Hq * a.nQ;
+  attn_bwd_dq_kernel<D><<<a.n_units < sms ? a.n_units : sms, kBwdThreads, L::kSmemBytes, st>>>(mq, mk, mv, mdo, a);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Sq) {
+  if (B <= 0 || Hq <= 0 || Sq <= 0) return 0;
+  return ((size_t)B * Hq * Sq * sizeof(float) + 255) & ~size_t(255);
+}
+
+attn_status attn_bwd(const attn_bwd_params* p, void* workspace, size_t workspace_bytes, void* stream) {
+  using namespace attn_bwd_kernels;
+  if (!p) return ATTN_ERR_INVALID_ARG;
+  if (p->B < 0 || p->Sq < 0 || p->Skv < 0 || p->Hq <= 0 || p->Hkv <= 0) return ATTN_ERR_INVALID_ARG;
+  if (p->Hq % p->Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (p->D != 64 && p->D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (p->mask.kind != ATTN_MASK_NONE && p->mask.kind != ATTN_MASK_CAUSAL && p->mask.kind != ATTN_MASK_WINDOW)
+    return p->mask.kind == ATTN_MASK_DOCUMENT ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+  if (p->B == 0 || p->Sq == 0) return ATTN_OK;
+  if (!p->q || !p->o || !p->dout || !p->lse || !p->dq || (p->Skv > 0 && (!p->k || !p->v || !p->dk || !p->dv)))
+    return ATTN_ERR_INVALID_ARG;
+  const void* ptrs[] = {p->q, p->k, p->v, p->o, p->dout, p->dq, p->dk, p->dv};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return ATTN_ERR_UNSUPPORTED;
+  const int64_t* strides[] = {p->q_stride, p->k_stride, p->v_stride, p->o_stride,
+                              p->do_stride, p->dq_stride, p->dk_stride, p->dv_stride};
+  for (const int64_t* st : strides)
+    if (!strides_ok(st, 3)) return ATTN_ERR_UNSUPPORTED;
+  const size_t need = attn_bwd_workspace_bytes(p->B, p->Hq, p->Sq);
+  if (!workspace || !aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // rowsum(dO o O) per (b, h, i)
+  DeltaArgs da;
+  da.o = static_cast<const __nv_bfloat16*>(p->o);
+  da.dout = static_cast<const __nv_bfloat16*>(p->dout);
+  da.o_sb = p->o_stride[0];
+  da.o_ss = p->o_stride[1];
+  da.o_sh = p->o_stride[2];
+  da.do_sb = p->do_stride[0];
+  da.do_ss = p->do_stride[1];
+  da.do_sh = p->do_stride[2];
+  da.B = p->B;
+  da.Hq = p->Hq;
+  da.Sq = p->Sq;
+  da.D = p->D;
+  da.delta = static_cast<float*>(workspace);
+  const int64_t rows = (int64_t)p->B * p->Hq * p->Sq;
+  if ((rows + 7) / 8 > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+  delta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(da);
+
+  BwdArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.Sq = p->Sq;
+  a.Skv = p->Skv;
+  a.g = p->Hq / p->Hkv;
+  a.scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
+  a.scale_log2 = a.scale * kLog2e;
+  a.mask = p->mask.kind;
+  a.q_offset = p->mask.kind == ATTN_MASK_NONE ? 0 : p->mask.q_offset;
+  a.wl = p->mask.kind == ATTN_MASK_WINDOW ? (p->mask.window_left < 0 ? -1 : p->mask.window_left) : -1;
+  a.wr = p->mask.kind == ATTN_MASK_CAUSAL ? 0
+                                           : (p->mask.kind == ATTN_MASK_WINDOW
+                                                  ? (p->mask.window_right < 0 ? -1 : p->mask.window_right)
+                                                  : -1);
+  a.nQ = (p->Sq + kTile - 1) / kTile;
+  a.nK = (p->Skv + kTile - 1) / kTile;
+  a.lse = p->lse;
+  a.delta = static_cast<const float*>(workspace);
+  a.dq = static_cast<__nv_bfloat16*>(p->dq);
+  a.dk = static_cast<__nv_bfloat16*>(p->dk);
+  a.dv = static_cast<__nv_bfloat16*>(p->dv);
+  a.dq_sb = p->dq_stride[0];
+  a.dq_ss = p->dq_stride[1];
+  a.dq_sh = p->dq_stride[2];
+  a.dk_sb = p->dk_stride[0];
+  a.dk_ss = p->dk_stride[1];
+  a.dk_sh = p->dk_stride[2];
+  a.dv_sb = p->dv_stride[0];
+  a.dv_ss = p->dv_stride[1];
+  a.dv_sh = p->dv_stride[2];
+  a.status = p->status;
+  if ((long)a.B * a.Hq * a.nQ > 0x7fffffffL || (long)a.B * a.Hkv * a.nK > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+
+  CUtensorMap mq, mk, mv, mdo;
+  const uint64_t dq[4] = {(uint64_t)p->D, (uint64_t)p->Sq, (uint64_t)p->Hq, (uint64_t)p->B};
+  const uint64_t dk[4] = {(uint64_t)p->D, (uint64_t)(p->Skv > 0 ? p->Skv : 1), (uint64_t)p->Hkv, (uint64_t)p->B};
+  int64_t sq[3], sk[3], sv[3], sdo[3];
+  if (!map_strides(p->q_stride, dq, sq) || !map_strides(p->do_stride, dq, sdo) ||
+      (p->Skv > 0 && (!map_strides(p->k_stride, dk, sk) || !map_strides(p->v_stride, dk, sv))))
+    return ATTN_ERR_UNSUPPORTED;
+  if (p->Skv == 0) {
+    for (int i = 0; i < 3; ++i) sk[i] = sv[i] = sq[i];
+  }
+  if (attn_status e = make_map(&mq, p->q, 4, dq, sq, kTile, 1)) return e;
+  if (attn_status e = make_map(&mdo, p->dout, 4, dq, sdo, kTile, 1)) return e;
+  // With Skv == 0 no key tile is ever loaded; the unused maps point at Q.
+  if (attn_status e = make_map(&mk, p->Skv > 0 ? p->k : p->q, 4, p->Skv > 0 ? dk : dq, sk, kTile, 1)) return e;
+  if (attn_status e = make_map(&mv, p->Skv > 0 ? p->v : p->q, 4, p->Skv > 0 ? dk : dq, sv, kTile, 1)) return e;
+  return p->D == 128 ? launch_bwd<128>(mq, mk, mv, mdo, a, st) : launch_bwd<64>(mq, mk, mv, mdo, a, st);
+}
 
 const char* attn_status_str(attn_status s) {
   switch (s) {

@@ -1,0 +1,793 @@
+// bwd_kernel.cuh - attention backward for sm_100a (attn_bwd): dQ, dK, dV of
+// O = softmax(scale * Q K^T + mask) V for an upstream gradient dO, with the
+// forward's log-sum-exp as input. The FlashAttention overview ("Examples")
+// names this backward pass and its deterministic option; the kernels here
+// are deterministic by construction: every output element is accumulated by
+// one CTA in a fixed order, with no atomics.
+//
+// With P = exp(scale * S - LSE) (S = Q K^T, masked entries 0), the chain rule
+// gives dV = P^T dO, dP = dO V^T, dS = P o (dP - delta) with delta_i =
+// dO_i . O_i, dQ = scale * dS K and dK = scale * dS^T Q. Three kernels:
+//   delta_kernel   delta_i for every (b, h, i) on CUDA cores;
+//   dkdv kernel    one work unit per (b, KV head, 128-key tile): loops over
+//                  every query tile and every query head of the group,
+//                  recomputing S^T = K Q^T and dP^T = V dO^T in TMEM, writing
+//                  P^T and dS^T back to TMEM as bf16 and accumulating
+//                  dV += P^T dO and dK += dS^T Q there (tcgen05, A from TMEM);
+//   dq kernel      one work unit per (b, query head, 128-row tile): loops over
+//                  the key tiles, S = Q K^T and dP = dO V^T in TMEM, dS back
+//                  to TMEM as bf16, dQ += dS K.
+// Warp roles (256 threads): warps 0-3 compute (thread = TMEM lane = key row
+// in dkdv, query row in dq), warp 4 MMA issue (owns TMEM), warp 5 TMA
+// producer, warps 6-7 idle. Every wait is bounded (sm100.cuh).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+
+namespace attn_bwd_kernels {
+
+using namespace attn_sm100;
+
+constexpr int kTile = 128;  // rows of a Q tile, keys of a K/V tile
+constexpr int kBwdThreads = 256;
+constexpr int kBMmaWarp = 4;
+constexpr int kBTmaWarp = 5;
+constexpr float kLog2eB = 1.4426950408889634f;
+enum : int { BMASK_NONE = 0, BMASK_CAUSAL = 1, BMASK_WINDOW = 2 };
+enum : int { BDEV_TIMEOUT = 1 };
+
+struct BwdArgs {
+  int B, Hq, Hkv, Sq, Skv, g;
+  float scale, scale_log2;
+  int mask, wl, wr, q_offset;  // window form: q_pos - wl <= key <= q_pos + wr (-1 = unbounded side)
+  int nQ, nK;
+  const float* lse;    // [B][Hq][Sq] natural log (from the forward)
+  const float* delta;  // [B][Hq][Sq] (workspace, written by delta_kernel)
+  __nv_bfloat16 *dq, *dk, *dv;
+  int64_t dq_sb, dq_ss, dq_sh, dk_sb, dk_ss, dk_sh, dv_sb, dv_ss, dv_sh;
+  int n_units;
+  int* status;
+};
+
+// ---------------------------------------------------------------- delta
+// delta[b][h][i] = sum_d dO[b,i,h,d] * O[b,i,h,d]; one warp per row.
+struct DeltaArgs {
+  const __nv_bfloat16 *o, *dout;
+  int64_t o_sb, o_ss, o_sh, do_sb, do_ss, do_sh;
+  int B, Hq, Sq, D;
+  float* delta;
+};
+
+__global__ void __launch_bounds__(256) delta_kernel(const DeltaArgs a) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= (int64_t)a.B * a.Hq * a.Sq) return;
+  const int i = (int)(row % a.Sq);
+  const int h = (int)((row / a.Sq) % a.Hq);
+  const int b = (int)(row / ((int64_t)a.Sq * a.Hq));
+  const __nv_bfloat16* o = a.o + b * a.o_sb + (int64_t)i * a.o_ss + (int64_t)h * a.o_sh;
+  const __nv_bfloat16* d = a.dout + b * a.do_sb + (int64_t)i * a.do_ss + (int64_t)h * a.do_sh;
+  float acc = 0.f;
+  for (int c = 2 * lane; c < a.D; c += 64) {
+    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + c));
+    const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(d + c));
+    acc = fmaf(x.x, y.x, acc);
+    acc = fmaf(x.y, y.y, acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) a.delta[((int64_t)b * a.Hq + h) * a.Sq + i] = acc;
+}
+
+// ---------------------------------------------------------------- masks
+// Query tiles [lo, hi] that meet key tile t (keys k0..k1) under the window
+// form; false when none.
+__device__ __forceinline__ bool q_range_for_k(const BwdArgs& a, int t, int& lo, int& hi) {
+  const long k0 = (long)t * kTile, k1 = min((long)(t + 1) * kTile, (long)a.Skv) - 1;
+  long qlo = 0, qhi = (long)a.Sq - 1;
+  if (a.mask != BMASK_NONE) {
+    // key k is seen by q_pos in [k - wr, k + wl]; q_pos = i + q_offset
+    if (a.wr >= 0) qlo = max(qlo, k0 - a.wr - a.q_offset);
+    if (a.wl >= 0) qhi = min(qhi, k1 + a.wl - a.q_offset);
+  }
+  if (qhi < qlo) return false;
+  lo = (int)(qlo / kTile);
+  hi = (int)(qhi / kTile);
+  return true;
+}
+
+// Key tiles [lo, hi] that meet query tile qt.
+__device__ __forceinline__ bool k_range_for_q(const BwdArgs& a, int qt, int& lo, int& hi) {
+  const long q0 = (long)qt * kTile + a.q_offset, q1 = min((long)(qt + 1) * kTile, (long)a.Sq) - 1 + a.q_offset;
+  long klo = 0, khi = (long)a.Skv - 1;
+  if (a.mask != BMASK_NONE) {
+    if (a.wl >= 0) klo = max(klo, q0 - a.wl);
+    if (a.wr >= 0) khi = min(khi, q1 + a.wr);
+  }
+  if (khi < klo) return false;
+  lo = (int)(klo / kTile);
+  hi = (int)(khi / kTile);
+  return true;
+}
+
+// A (query tile qt, key tile t) pair needs per-element masking unless every
+// in-tile pair is allowed and neither side is ragged.
+__device__ __forceinline__ bool pair_full(const BwdArgs& a, int qt, int t) {
+  const long q0 = (long)qt * kTile, q1 = (long)(qt + 1) * kTile - 1;
+  const long k0 = (long)t * kTile, k1 = (long)(t + 1) * kTile - 1;
+  if (q1 >= a.Sq || k1 >= a.Skv) return false;
+  if (a.mask == BMASK_NONE) return true;
+  bool full = true;
+  if (a.wl >= 0 && k0 < q1 + a.q_offset - a.wl) full = false;
+  if (a.wr >= 0 && k1 > q0 + a.q_offset + a.wr) full = false;
+  return full;
+}
+
+// Bit e of the result: element e of a 32-wide chunk starting at position
+// c0 on the other axis is allowed, given that the thread's own position is
+// allowed exactly for other-axis positions in [lo, hi].
+__device__ __forceinline__ uint32_t range_bits(long lo, long hi, long c0) {
+  const long a = lo - c0, b = hi - c0;
+  if (b < 0 || a > 31 || b < a) return 0u;
+  const int l = (int)max(a, 0l), h = (int)min(b, 31l);
+  return (0xffffffffu >> (31 - h)) & (0xffffffffu << l);
+}
+
+// ---------------------------------------------------------------- layout
+template <int D>
+struct BLayout {
+  static constexpr int kTileBytes = kTile * D * 2;    // one operand tile (128 rows x D bf16)
+  static constexpr int kChunk = kTile * 64 * 2;       // one 128-row x 64-column SW128 box
+  // dkdv: K, V of the unit, then a 2-slot ring of (Q, dO, lse, delta) per step.
+  // dq: Q, dO of the unit, then a 2-slot ring of (K, V) per step.
+  static constexpr int kFixOff = 0;                   // two unit tiles
+  static constexpr int kRingOff = 2 * kTileBytes;     // 2 slots x two step tiles
+  static constexpr int kVecOff = kRingOff + 4 * kTileBytes;  // dkdv: 2 slots x (lse, delta) x 128 floats
+  static constexpr int kBarOff = kVecOff + 2 * 2 * kTile * 4;
+  // Each CTA allocates all 512 TMEM columns, so two CTAs must never share an
+  // SM: the request is padded past half of the SM's 228 KB of shared memory.
+  static constexpr int kUsedBytes = kBarOff + 1024 + 1024;
+  static constexpr int kSmemBytes = kUsedBytes > 120 * 1024 ? kUsedBytes : 120 * 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+  static_assert(kVecOff % 1024 == 0, "operand tiles stay 1024-byte aligned");
+};
+
+struct BBarriers {
+  uint64_t fix_full, fix_empty;  // unit tiles loaded / released
+  uint64_t ring_full[2], ring_empty[2];
+  uint64_t mm1_ready;   // the step's first two products (S / dP) are in TMEM
+  uint64_t comp_ready;  // the compute warps wrote P^T / dS^T (dkdv) or dS (dq): 128 arrivals
+  uint64_t acc_done;    // the unit's accumulators are final
+  uint64_t acc_free;    // the epilogue read them: 128 arrivals
+  uint64_t vec_ready[2];  // dkdv: the step's LSE / delta columns are in shared memory (128 arrivals)
+  uint64_t final_mma;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// ---------------------------------------------------------------- work maps
+// dkdv unit u -> (b, hk, key tile t); t ascending is heaviest first for the
+// causal form. Steps: q tiles qt of [lo, hi] times the g query heads.
+struct KvUnit {
+  int b, hk, t, qlo, n;  // n = steps
+};
+__device__ __forceinline__ KvUnit kv_unit(const BwdArgs& a, int u) {
+  KvUnit w;
+  const int per = a.B * a.Hkv;
+  w.t = u / per;
+  const int r = u % per;
+  w.b = r / a.Hkv;
+  w.hk = r % a.Hkv;
+  int lo = 0, hi = -1;
+  w.n = q_range_for_k(a, w.t, lo, hi) ? (hi - lo + 1) * a.g : 0;
+  w.qlo = lo;
+  return w;
+}
+// dq unit u -> (b, h, q tile qt); last q tiles first (the most key tiles).
+struct QUnit {
+  int b, h, qt, klo, n;
+};
+__device__ __forceinline__ QUnit q_unit(const BwdArgs& a, int u) {
+  QUnit w;
+  const int per = a.B * a.Hq;
+  w.qt = a.nQ - 1 - u / per;
+  const int r = u % per;
+  w.b = r / a.Hq;
+  w.h = r % a.Hq;
+  int lo = 0, hi = -1;
+  w.n = k_range_for_q(a, w.qt, lo, hi) ? hi - lo + 1 : 0;
+  w.klo = lo;
+  return w;
+}
+
+__device__ __forceinline__ float bex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------- dK / dV
+// TMEM columns: S^T [0, 128), dP^T [128, 256), dV [256, 256 + D), dK [256 + D, 256 + 2D).
+// P^T (bf16 pairs) replaces the first 64 columns of S^T, dS^T the first 64 of dP^T.
+// MMA order per step: S^T, dP^T | (compute) | dV, dK, S^T(next), dP^T(next).
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                         const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
+                         const BwdArgs a) {
+  using L = BLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  BBarriers& bar = *reinterpret_cast<BBarriers*>(smem + L::kBarOff);
+  const int warp = threadIdx.x / 32;
+  volatile int* abort_flag = &bar.abort_flag;
+  if (threadIdx.x == 0) {
+    bar.abort_flag = 0;
+    mbar_init(&bar.fix_full, 1);
+    mbar_init(&bar.fix_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar.ring_full[i], 1);
+      mbar_init(&bar.ring_empty[i], 1);
+    }
+    mbar_init(&bar.mm1_ready, 1);
+    mbar_init(&bar.comp_ready, kTile);
+    mbar_init(&bar.acc_done, 1);
+    mbar_init(&bar.acc_free, kTile);
+    mbar_init(&bar.vec_ready[0], kTile);
+    mbar_init(&bar.vec_ready[1], kTile);
+    mbar_init(&bar.final_mma, 1);
+    fence_barrier_init();
+  }
+  if (warp == kBMmaWarp) {
+    tmem_alloc(&bar.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  const int G = gridDim.x;
+  const int rounds = (a.n_units + G - 1) / G;
+  auto unit_of = [&](int r) -> int {
+    const int c = (r & 1) ? G - 1 - (int)blockIdx.x : (int)blockIdx.x;
+    const int u = r * G + c;
+    return u < a.n_units ? u : -1;
+  };
+  auto wait_all = [&](uint64_t* b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag)); };
+  auto wait_spin_all = [&](uint64_t* b, uint32_t par) {
+    return __all_sync(0xffffffffu, mbar_wait_spin(b, par, abort_flag));
+  };
+  // step s of a unit: q tile qlo + s / g, query head hk * g + s % g
+  if (warp == kBTmaWarp) {
+    // ------------------------------------------------------------ producer
+    if (elect_one_sync()) {
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_do);
+    }
+    __syncwarp();
+    int ucnt = 0, gstep = 0;
+    bool ok = true;
+    for (int r = 0; ok && r < rounds; ++r) {
+      const int u = unit_of(r);
+      if (u < 0) continue;
+      const KvUnit w = kv_unit(a, u);
+      if (w.n == 0) continue;
+      if (ucnt > 0 && !wait_all(&bar.fix_empty, (ucnt - 1) & 1)) { ok = false; break; }
+      if (elect_one_sync()) {
+        mbar_arrive_expect_tx(&bar.fix_full, 2 * L::kTileBytes);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_4d(smem + L::kFixOff + c * L::kChunk, &map_k, &bar.fix_full, c * 64, w.t * kTile, w.hk, w.b);
+          tma_load_4d(smem + L::kFixOff + L::kTileBytes + c * L::kChunk, &map_v, &bar.fix_full, c * 64, w.t * kTile,
+                      w.hk, w.b);
+        }
+      }
+      __syncwarp();
+      ++ucnt;
+      for (int s = 0; s < w.n; ++s, ++gstep) {
+        const int slot = gstep & 1, use = gstep >> 1;
+        if (use > 0 && !wait_all(&bar.ring_empty[slot], (use - 1) & 1)) { ok = false; break; }
+        const int qt = w.qlo + s / a.g, h = w.hk * a.g + s % a.g;
+        if (elect_one_sync()) {
+          uint64_t* fb = &bar.ring_full[slot];
+          mbar_arrive_expect_tx(fb, 2 * L::kTileBytes);
+          uint8_t* base = smem + L::kRingOff + slot * 2 * L::kTileBytes;
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_4d(base + c * L::kChunk, &map_q, fb, c * 64, qt * kTile, h, w.b);
+            tma_load_4d(base + L::kTileBytes + c * L::kChunk, &map_do, fb, c * 64, qt * kTile, h, w.b);
+          }
+        }
+        __syncwarp();
+      }
+    }
+    if (*abort_flag) {
+      if (ucnt > 0) mbar_wait_timeout(&bar.fix_full, (ucnt - 1) & 1);
+      for (int k = max(0, gstep - 2); k < gstep; ++k) mbar_wait_timeout(&bar.ring_full[k & 1], (k >> 1) & 1);
+    }
+  } else if (warp == kBMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    constexpr uint32_t kHi = sdesc_sw128_hi(1024);
+    constexpr uint32_t idesc_mm1 = idesc_bf16_f32(128, 128, 0, 0);  // K-major A and B
+    constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);    // B MN-major (rows x D tiles)
+    constexpr uint32_t kTileUnits = L::kTileBytes >> 4;
+    const uint32_t k_lo = sdesc_sw128_lo(smem_u32(smem + L::kFixOff), 16);
+    const uint32_t v_lo = k_lo + kTileUnits;
+    const uint32_t ring_lo = sdesc_sw128_lo(smem_u32(smem + L::kRingOff), 16);
+    const uint32_t ring_mn = sdesc_sw128_lo(smem_u32(smem + L::kRingOff), L::kChunk);
+    // S^T = K Q^T into [0, 128) and dP^T = V dO^T into [128, 256) for ring slot `slot`.
+    auto mm1 = [&](int slot) {
+      const uint32_t qa = ring_lo + (uint32_t)slot * 2 * kTileUnits, da = qa + kTileUnits;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
+        mma_ss(tmem, sdesc_join(k_lo + off, kHi), sdesc_join(qa + off, kHi), idesc_mm1, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
+        mma_ss(tmem + 128, sdesc_join(v_lo + off, kHi), sdesc_join(da + off, kHi), idesc_mm1, kk > 0);
+      }
+      mma_commit(&bar.mm1_ready);
+    };
+    int ucnt = 0, gstep = 0;
+    bool ok = true;
+    for (int r = 0; ok && r < rounds; ++r) {
+      const int u = unit_of(r);
+      if (u < 0) continue;
+      const KvUnit w = kv_unit(a, u);
+      if (w.n == 0) continue;
+      ok = wait_all(&bar.fix_full, ucnt & 1) && wait_all(&bar.ring_full[gstep & 1], (gstep >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one_sync()) mm1(gstep & 1);
+      __syncwarp();
+      for (int s = 0; s < w.n; ++s) {
+        const int g = gstep + s, slot = g & 1;
+        const bool more = s + 1 < w.n;
+        if (more && !wait_all(&bar.ring_full[(g + 1) & 1], ((g + 1) >> 1) & 1)) { ok = false; break; }
+        if (!wait_spin_all(&bar.comp_ready, g & 1)) { ok = false; break; }
+        // The unit's first accumulation overwrites dV / dK: the previous
+        // unit's epilogue must have read them.
+        if (s == 0 && ucnt > 0 && !wait_all(&bar.acc_free, (ucnt - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one_sync()) {
+          const uint32_t qmn = ring_mn + (uint32_t)slot * 2 * kTileUnits, dmn = qmn + kTileUnits;
+          // dV += P^T dO: P^T from TMEM columns [0, 64), dO rows 16kk..
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + 256, tmem + kk * 8, sdesc_join(dmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
+                   (s > 0 || kk > 0) ? 1u : 0u);
+          // dK += dS^T Q: dS^T from TMEM columns [128, 192)
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + 256 + D, tmem + 128 + kk * 8, sdesc_join(qmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
+                   (s > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bar.ring_empty[slot]);
+          if (!more) {
+            mma_commit(&bar.acc_done);
+            mma_commit(&bar.fix_empty);
+          } else {
+            mm1((g + 1) & 1);
+          }
+        }
+        __syncwarp();
+      }
+      gstep += w.n;
+      ++ucnt;
+    }
+    if (elect_one_sync()) mma_commit(&bar.final_mma);
+    __syncwarp();
+    mbar_wait_timeout(&bar.final_mma, 0);
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ compute
+    const int row = threadIdx.x;  // key row of the tile = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    int ucnt = 0, gstep = 0;
+    bool ok = true;
+    const float NEG_INF = -__int_as_float(0x7f800000);
+    for (int r = 0; ok && r < rounds; ++r) {
+      const int u = unit_of(r);
+      if (u < 0) continue;
+      const KvUnit w = kv_unit(a, u);
+      const long key = (long)w.t * kTile + row;
+      if (w.n == 0) {
+        // no query sees these keys: their gradients are exactly zero
+        if (key < a.Skv) {
+          __nv_bfloat16* dvr = a.dv + w.b * a.dv_sb + key * a.dv_ss + (int64_t)w.hk * a.dv_sh;
+          __nv_bfloat16* dkr = a.dk + w.b * a.dk_sb + key * a.dk_ss + (int64_t)w.hk * a.dk_sh;
+          for (int c = 0; c < D; c += 8) {
+            *reinterpret_cast<uint4*>(dvr + c) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(dkr + c) = make_uint4(0, 0, 0, 0);
+          }
+        }
+        continue;
+      }
+      for (int s = 0; s < w.n; ++s) {
+        const int g = gstep + s, slot = g & 1;
+        const int qt = w.qlo + s / a.g, h = w.hk * a.g + s % a.g;
+        // Column values of the step (LSE and delta of the q tile's queries):
+        // thread r fetches query qt*128 + r into a shared, double-buffered
+        // array; a bounded mbarrier (128 arrivals) publishes it.
+        float* vec = reinterpret_cast<float*>(smem + L::kVecOff) + slot * 2 * kTile;
+        {
+          const int qi = qt * kTile + row;
+          float lv = NEG_INF, dv = 0.f;
+          if (qi < a.Sq) {
+            const int64_t ix = ((int64_t)w.b * a.Hq + h) * a.Sq + qi;
+            lv = a.lse[ix];
+            dv = a.delta[ix];
+          }
+          vec[row] = lv;
+          vec[kTile + row] = dv;
+          mbar_arrive(&bar.vec_ready[slot]);
+        }
+        if (!wait_spin_all(&bar.mm1_ready, g & 1)) { ok = false; break; }
+        if (!wait_spin_all(&bar.vec_ready[slot], (g >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const bool full = pair_full(a, qt, w.t);
+        // queries that see this key: q_pos in [key - wr, key + wl], q_pos = i + q_offset
+        long qlo_i = 0, qhi_i = (long)a.Sq - 1;
+        if (a.mask != BMASK_NONE) {
+          if (a.wr >= 0) qlo_i = max(qlo_i, key - a.wr - a.q_offset);
+          if (a.wl >= 0) qhi_i = min(qhi_i, key + a.wl - a.q_offset);
+        }
+        if (key >= a.Skv) qhi_i = -1;
+#pragma unroll 1
+        for (int c = 0; c < kTile / 32; ++c) {
+          float x[32], dp[32];
+          tmem_ld32f(lane_base + 32 * c, x);
+          tmem_ld32f(lane_base + 128 + 32 * c, dp);
+          tmem_ld_wait();
+          reg_fence_f<32>(x);
+          reg_fence_f<32>(dp);
+          const uint32_t bits = full ? 0xffffffffu : range_bits(qlo_i, qhi_i, (long)qt * kTile + 32 * c);
+          uint32_t pk[16], dk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float pe[2], de[2];
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+              const int col = 32 * c + e + z;
+              // LSE -inf (a row with no allowed key): no pair of it is allowed either
+              const float l2 = vec[col] == NEG_INF ? __int_as_float(0x7f800000) : vec[col] * kLog2eB;
+              const bool on = (bits >> (e + z)) & 1u;
+              const float p = on ? bex2(fmaf(x[e + z], a.scale_log2, -l2)) : 0.f;
+              pe[z] = p;
+              de[z] = p * (dp[e + z] - vec[kTile + col]);
+            }
+            pk[e / 2] = pack_bf16x2(pe[0], pe[1]);
+            dk[e / 2] = pack_bf16x2(de[0], de[1]);
+          }
+          // P^T chunk c -> columns [16c, 16c + 16) (S^T columns already read),
+          // dS^T chunk c -> [128 + 16c, 128 + 16c + 16) likewise
+          tmem_st16(lane_base + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(pk));
+          tmem_st16(lane_base + 128 + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(dk));
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar.comp_ready);
+      }
+      if (!ok) break;
+      // epilogue: dV, dK (x scale) rows -> bf16
+      if (!wait_all(&bar.acc_done, ucnt & 1)) break;
+      tc_fence_after();
+      {
+        // tcgen05.ld is warp-collective: every lane loads, only rows of real
+        // keys are stored (a ragged tile splits a warp).
+        const bool real = key < a.Skv;
+        __nv_bfloat16* dvr = a.dv + w.b * a.dv_sb + (real ? key : 0) * a.dv_ss + (int64_t)w.hk * a.dv_sh;
+        __nv_bfloat16* dkr = a.dk + w.b * a.dk_sb + (real ? key : 0) * a.dk_ss + (int64_t)w.hk * a.dk_sh;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          float v0[32], k0[32];
+          tmem_ld32f(lane_base + 256 + c, v0);
+          tmem_ld32f(lane_base + 256 + D + c, k0);
+          tmem_ld_wait();
+          reg_fence_f<32>(v0);
+          reg_fence_f<32>(k0);
+#pragma unroll
+          for (int e = 0; real && e < 32; e += 8) {
+            uint4 pv, pkk;
+            pv.x = pack_bf16x2(v0[e], v0[e + 1]);
+            pv.y = pack_bf16x2(v0[e + 2], v0[e + 3]);
+            pv.z = pack_bf16x2(v0[e + 4], v0[e + 5]);
+            pv.w = pack_bf16x2(v0[e + 6], v0[e + 7]);
+            pkk.x = pack_bf16x2(k0[e] * a.scale, k0[e + 1] * a.scale);
+            pkk.y = pack_bf16x2(k0[e + 2] * a.scale, k0[e + 3] * a.scale);
+            pkk.z = pack_bf16x2(k0[e + 4] * a.scale, k0[e + 5] * a.scale);
+            pkk.w = pack_bf16x2(k0[e + 6] * a.scale, k0[e + 7] * a.scale);
+            *reinterpret_cast<uint4*>(dvr + c + e) = pv;
+            *reinterpret_cast<uint4*>(dkr + c + e) = pkk;
+          }
+          __syncwarp();  // reconverge before the next warp-collective load
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar.acc_free);
+      gstep += w.n;
+      ++ucnt;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kBMmaWarp) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && bar.abort_flag && a.status) atomicOr(a.status, BDEV_TIMEOUT);
+}
+
+// ---------------------------------------------------------------- dQ
+// TMEM columns: S [0, 128), dP [128, 256), dQ [256, 256 + D). dS (bf16 pairs)
+// replaces the first 64 columns of S. MMA order per step:
+// S, dP | (compute) | dQ, S(next), dP(next).
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                       const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
+                       const BwdArgs a) {
+  using L = BLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  BBarriers& bar = *reinterpret_cast<BBarriers*>(smem + L::kBarOff);
+  const int warp = threadIdx.x / 32;
+  volatile int* abort_flag = &bar.abort_flag;
+  if (threadIdx.x == 0) {
+    bar.abort_flag = 0;
+    mbar_init(&bar.fix_full, 1);
+    mbar_init(&bar.fix_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar.ring_full[i], 1);
+      mbar_init(&bar.ring_empty[i], 1);
+    }
+    mbar_init(&bar.mm1_ready, 1);
+    mbar_init(&bar.comp_ready, kTile);
+    mbar_init(&bar.acc_done, 1);
+    mbar_init(&bar.acc_free, kTile);
+    mbar_init(&bar.final_mma, 1);
+    fence_barrier_init();
+  }
+  if (warp == kBMmaWarp) {
+    tmem_alloc(&bar.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar.tmem_base;
+  const int G = gridDim.x;
+  const int rounds = (a.n_units + G - 1) / G;
+  auto unit_of = [&](int r) -> int {
+    const int c = (r & 1) ? G - 1 - (int)blockIdx.x : (int)blockIdx.x;
+    const int u = r * G + c;
+    return u < a.n_units ? u : -1;
+  };
+  auto wait_all = [&](uint64_t* b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag)); };
+  auto wait_spin_all = [&](uint64_t* b, uint32_t par) {
+    return __all_sync(0xffffffffu, mbar_wait_spin(b, par, abort_flag));
+  };
+  if (warp == kBTmaWarp) {
+    // ------------------------------------------------------------ producer
+    if (elect_one_sync()) {
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+    }
+    __syncwarp();
+    int ucnt = 0, gstep = 0;
+    bool ok = true;
+    for (int r = 0; ok && r < rounds; ++r) {
+      const int u = unit_of(r);
+      if (u < 0) continue;
+      const QUnit w = q_unit(a, u);
+      if (w.n == 0) continue;
+      const int hk = w.h / a.g;
+      if (ucnt > 0 && !wait_all(&bar.fix_empty, (ucnt - 1) & 1)) { ok = false; break; }
+      if (elect_one_sync()) {
+        mbar_arrive_expect_tx(&bar.fix_full, 2 * L::kTileBytes);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_4d(smem + L::kFixOff + c * L::kChunk, &map_q, &bar.fix_full, c * 64, w.qt * kTile, w.h, w.b);
+          tma_load_4d(smem + L::kFixOff + L::kTileBytes + c * L::kChunk, &map_do, &bar.fix_full, c * 64,
+                      w.qt * kTile, w.h, w.b);
+        }
+      }
+      __syncwarp();
+      ++ucnt;
+      for (int s = 0; s < w.n; ++s, ++gstep) {
+        const int slot = gstep & 1, use = gstep >> 1;
+        if (use > 0 && !wait_all(&bar.ring_empty[slot], (use - 1) & 1)) { ok = false; break; }
+        const int t = w.klo + s;
+        if (elect_one_sync()) {
+          uint64_t* fb = &bar.ring_full[slot];
+          mbar_arrive_expect_tx(fb, 2 * L::kTileBytes);
+          uint8_t* base = smem + L::kRingOff + slot * 2 * L::kTileBytes;
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_4d(base + c * L::kChunk, &map_k, fb, c * 64, t * kTile, hk, w.b);
+            tma_load_4d(base + L::kTileBytes + c * L::kChunk, &map_v, fb, c * 64, t * kTile, hk, w.b);
+          }
+        }
+        __syncwarp();
+      }
+    }
+    if (*abort_flag) {
+      if (ucnt > 0) mbar_wait_timeout(&bar.fix_full, (ucnt - 1) & 1);
+      for (int k = max(0, gstep - 2); k < gstep; ++k) mbar_wait_timeout(&bar.ring_full[k & 1], (k >> 1) & 1);
+    }
+  } else if (warp == kBMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    constexpr uint32_t kHi = sdesc_sw128_hi(1024);
+    constexpr uint32_t idesc_mm1 = idesc_bf16_f32(128, 128, 0, 0);
+    constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
+    constexpr uint32_t kTileUnits = L::kTileBytes >> 4;
+    const uint32_t q_lo = sdesc_sw128_lo(smem_u32(smem + L::kFixOff), 16);
+    const uint32_t do_lo = q_lo + kTileUnits;
+    const uint32_t ring_lo = sdesc_sw128_lo(smem_u32(smem + L::kRingOff), 16);
+    const uint32_t ring_mn = sdesc_sw128_lo(smem_u32(smem + L::kRingOff), L::kChunk);
+    // S = Q K^T into [0, 128) and dP = dO V^T into [128, 256) for ring slot `slot`.
+    auto mm1 = [&](int slot) {
+      const uint32_t ka = ring_lo + (uint32_t)slot * 2 * kTileUnits, va = ka + kTileUnits;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
+        mma_ss(tmem, sdesc_join(q_lo + off, kHi), sdesc_join(ka + off, kHi), idesc_mm1, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
+        mma_ss(tmem + 128, sdesc_join(do_lo + off, kHi), sdesc_join(va + off, kHi), idesc_mm1, kk > 0);
+      }
+      mma_commit(&bar.mm1_ready);
+    };
+    int ucnt = 0, gstep = 0;
+    bool ok = true;
+    for (int r = 0; ok && r < rounds; ++r) {
+      const int u = unit_of(r);
+      if (u < 0) continue;
+      const QUnit w = q_unit(a, u);
+      if (w.n == 0) continue;
+      ok = wait_all(&bar.fix_full, ucnt & 1) && wait_all(&bar.ring_full[gstep & 1], (gstep >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one_sync()) mm1(gstep & 1);
+      __syncwarp();
+      for (int s = 0; s < w.n; ++s) {
+        const int g = gstep + s, slot = g & 1;
+        const bool more = s + 1 < w.n;
+        if (more && !wait_all(&bar.ring_full[(g + 1) & 1], ((g + 1) >> 1) & 1)) { ok = false; break; }
+        if (!wait_spin_all(&bar.comp_ready, g & 1)) { ok = false; break; }
+        if (s == 0 && ucnt > 0 && !wait_all(&bar.acc_free, (ucnt - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one_sync()) {
+          const uint32_t kmn = ring_mn + (uint32_t)slot * 2 * kTileUnits;
+          // dQ += dS K: dS from TMEM columns [0, 64), K rows 16kk..
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + 256, tmem + kk * 8, sdesc_join(kmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
+                   (s > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bar.ring_empty[slot]);
+          if (!more) {
+            mma_commit(&bar.acc_done);
+            mma_commit(&bar.fix_empty);
+          } else {
+            mm1((g + 1) & 1);
+          }
+        }
+        __syncwarp();
+      }
+      gstep += w.n;
+      ++ucnt;
+    }
+    if (elect_one_sync()) mma_commit(&bar.final_mma);
+    __syncwarp();
+    mbar_wait_timeout(&bar.final_mma, 0);
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ compute
+    const int row = threadIdx.x;  // query row of the tile = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const float NEG_INF = -__int_as_float(0x7f800000);
+    int ucnt = 0, gstep = 0;
+    bool ok = true;
+    for (int r = 0; ok && r < rounds; ++r) {
+      const int u = unit_of(r);
+      if (u < 0) continue;
+      const QUnit w = q_unit(a, u);
+      const int qi = w.qt * kTile + row;
+      const bool valid = qi < a.Sq;
+      if (w.n == 0) {
+        // these queries see no key: their gradient is exactly zero
+        if (valid) {
+          __nv_bfloat16* dqr = a.dq + w.b * a.dq_sb + (int64_t)qi * a.dq_ss + (int64_t)w.h * a.dq_sh;
+          for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(dqr + c) = make_uint4(0, 0, 0, 0);
+        }
+        continue;
+      }
+      const int64_t rix = ((int64_t)w.b * a.Hq + w.h) * a.Sq + min(qi, a.Sq - 1);
+      const float lse = a.lse[rix];
+      const float l2 = (!valid || lse == NEG_INF) ? __int_as_float(0x7f800000) : lse * kLog2eB;
+      const float dlt = a.delta[rix];
+      // keys this query sees: [q_pos - wl, q_pos + wr]
+      const long q_pos = (long)qi + a.q_offset;
+      long klo_i = 0, khi_i = (long)a.Skv - 1;
+      if (a.mask != BMASK_NONE) {
+        if (a.wl >= 0) klo_i = max(klo_i, q_pos - a.wl);
+        if (a.wr >= 0) khi_i = min(khi_i, q_pos + a.wr);
+      }
+      if (!valid) khi_i = -1;
+      for (int s = 0; s < w.n; ++s) {
+        const int g = gstep + s;
+        const int t = w.klo + s;
+        if (!wait_spin_all(&bar.mm1_ready, g & 1)) { ok = false; break; }
+        tc_fence_after();
+        const bool full = pair_full(a, w.qt, t);
+#pragma unroll 1
+        for (int c = 0; c < kTile / 32; ++c) {
+          float x[32], dp[32];
+          tmem_ld32f(lane_base + 32 * c, x);
+          tmem_ld32f(lane_base + 128 + 32 * c, dp);
+          tmem_ld_wait();
+          reg_fence_f<32>(x);
+          reg_fence_f<32>(dp);
+          const uint32_t bits = full ? 0xffffffffu : range_bits(klo_i, khi_i, (long)t * kTile + 32 * c);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float de[2];
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+              const bool on = (bits >> (e + z)) & 1u;
+              const float p = on ? bex2(fmaf(x[e + z], a.scale_log2, -l2)) : 0.f;
+              de[z] = p * (dp[e + z] - dlt);
+            }
+            pk[e / 2] = pack_bf16x2(de[0], de[1]);
+          }
+          // dS chunk c -> columns [16c, 16c + 16) (S columns already read)
+          tmem_st16(lane_base + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(pk));
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar.comp_ready);
+      }
+      if (!ok) break;
+      if (!wait_all(&bar.acc_done, ucnt & 1)) break;
+      tc_fence_after();
+      {
+        // tcgen05.ld is warp-collective: every lane loads, only real query rows are stored
+        __nv_bfloat16* dqr = a.dq + w.b * a.dq_sb + (int64_t)(valid ? qi : 0) * a.dq_ss + (int64_t)w.h * a.dq_sh;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          float q0[32];
+          tmem_ld32f(lane_base + 256 + c, q0);
+          tmem_ld_wait();
+          reg_fence_f<32>(q0);
+#pragma unroll
+          for (int e = 0; valid && e < 32; e += 8) {
+            uint4 pq;
+            pq.x = pack_bf16x2(q0[e] * a.scale, q0[e + 1] * a.scale);
+            pq.y = pack_bf16x2(q0[e + 2] * a.scale, q0[e + 3] * a.scale);
+            pq.z = pack_bf16x2(q0[e + 4] * a.scale, q0[e + 5] * a.scale);
+            pq.w = pack_bf16x2(q0[e + 6] * a.scale, q0[e + 7] * a.scale);
+            *reinterpret_cast<uint4*>(dqr + c + e) = pq;
+          }
+          __syncwarp();  // reconverge before the next warp-collective load
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar.acc_free);
+      gstep += w.n;
+      ++ucnt;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kBMmaWarp) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && bar.abort_flag && a.status) atomicOr(a.status, BDEV_TIMEOUT);
+}
+
+}  // namespace attn_bwd_kernels

@@ -236,6 +236,38 @@ attn_status attn_lse_combine(const float *o_parts, const float *lse_parts, int r
 #define ATTN_DECODE_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
 attn_status attn_decode_noalloc(const attn_decode_params *p, void *stream);
 
+/* Backward of attn_fwd (FlashAttention overview, "Examples": the backward
+ * pass of flash_attn_func and its `deterministic` option): dQ, dK, dV for the
+ * upstream gradient dO, from Q, K, V, the forward's O and LSE. With
+ * P = exp(scale * Q K^T - LSE) over the allowed pairs:
+ *   dV = P^T dO,  dS = P o (dO V^T - rowsum(dO o O)),  dQ = scale dS K,  dK = scale dS^T Q,
+ * with dK and dV summed over the query heads of each KV head (GQA/MQA).
+ * Three kernels: a row reduction for rowsum(dO o O) into the workspace, then
+ * one tcgen05 kernel over key tiles (dK, dV) and one over query tiles (dQ).
+ * Every output element is accumulated by one CTA in a fixed order with no
+ * atomics, so results are bit-identical from run to run whatever
+ * `deterministic` says (the flag is accepted for interface compatibility).
+ * Supported: masks NONE / CAUSAL / WINDOW, no score mod, D in {64, 128};
+ * anything else returns ATTN_ERR_UNSUPPORTED. Layout rules as for attn_fwd;
+ * `workspace` is caller-owned device memory of at least
+ * attn_bwd_workspace_bytes(B, Hq, Sq). Sq == 0 or B == 0 launches nothing;
+ * Skv == 0 gives dQ = 0 (dK, dV are empty). */
+typedef struct {
+  const void *q, *k, *v, *o, *dout;  /* bf16 [B][S][H][D] via the strides below */
+  const float *lse;                  /* fp32 [B][Hq][Sq] contiguous, natural log, from attn_fwd */
+  void *dq, *dk, *dv;                /* bf16 outputs, shaped like q, k, v */
+  int64_t q_stride[3], k_stride[3], v_stride[3], o_stride[3], do_stride[3];
+  int64_t dq_stride[3], dk_stride[3], dv_stride[3];
+  int B, Hq, Hkv, Sq, Skv, D;
+  float scale;                       /* <= 0 selects 1/sqrt(D) */
+  attn_mask_spec mask;               /* NONE, CAUSAL or WINDOW */
+  int deterministic;
+  int *status;                       /* optional device int, ATTN_DEV_* bits */
+} attn_bwd_params;
+
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Sq);
+attn_status attn_bwd(const attn_bwd_params *p, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Failure-detection self-test (no counterpart on the pages). Launches one
  * warp that waits, with the bounded wait every pipeline barrier of these
  * kernels uses, on a barrier nothing arrives on. After the wait's limit
