@@ -241,6 +241,38 @@ def prefill_setup(torch, ea, w: W.Prefill, device, seed_shift: int):
                 bm=bm, o=o, lse=lse)
 
 
+def backward_setup(torch, ea, w: W.Prefill, device, seed_shift: int):
+    """attn_bwd on a causal/window/no-mask prefill workload: the forward's O and
+    LSE plus a seeded upstream gradient dO, rotated over enough replicas that
+    the step's inputs exceed L2. Algorithmic FLOPs: the five products of the
+    chain rule (S, dP, dV, dK, dQ), 2.5x the forward's 4*D per pair."""
+    wr = W.Prefill(**{**w.__dict__, "seed": w.seed + seed_shift})
+    d = W.make_prefill_inputs(wr)
+    kw = {}
+    if w.mask == W.MASK_CAUSAL:
+        kw["causal"] = True
+    elif w.mask == W.MASK_WINDOW:
+        kw["window"] = (w.window_left, w.window_right)
+    q0, k0, v0 = (to_dev(d[x], device) for x in ("q", "k", "v"))
+    do0 = to_dev(W.normal_bf16(wr.seed + 0x200, (w.B, w.S, w.Hq, w.D)), device)
+    per_set = 2 * (3 * q0.numel() + 3 * k0.numel())  # q, o, dO, dq + k, v, dk, dv (bf16)
+    nrep = replicas_for(per_set)
+    sets = []
+    for r in range(nrep):
+        q, k, v, do = (x if r == 0 else x.clone() for x in (q0, k0, v0, do0))
+        o, lse = ea.attn_fwd(q, k, v, **kw)
+        sets.append((q, k, v, o, lse, do))
+    dq, dk, dv = torch.empty_like(q0), torch.empty_like(k0), torch.empty_like(v0)
+    ws = torch.empty(ea.load_library().attn_bwd_workspace_bytes(w.B, w.Hq, w.S), dtype=torch.uint8, device=device)
+    pairs = unmasked_pairs(w, d["doc_lens"])
+
+    def step(i):
+        q, k, v, o, lse, do = sets[i % nrep]
+        ea.attn_bwd(q, k, v, o, lse, do, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
+
+    return dict(step=step, pairs=pairs, flops=10 * w.D * pairs, nrep=nrep)
+
+
 def decode_setup(torch, ea, w: W.Decode, device, seed_shift: int):
     wr = W.Decode(**{**w.__dict__, "seed": w.seed + seed_shift})
     d = W.make_decode_inputs(wr)
@@ -519,7 +551,7 @@ def main():
     ap.add_argument("--workload", default=PRIMARY, choices=[k for k, v in W.WORKLOADS.items()
                                                           if isinstance(v, W.Prefill)])
     ap.add_argument("--secondary-steps", type=int, default=200)
-    ap.add_argument("--profile", default=None, choices=list(W.WORKLOADS) + ["block_mask"],
+    ap.add_argument("--profile", default=None, choices=list(W.WORKLOADS) + ["block_mask", "backward_" + PRIMARY],
                     help="run --steps eager steps of one workload (for ncu captures); prints no JSON line")
     ap.add_argument("--plumbing-check", action="store_true",
                     help="CPU only: rehearse the N-rank launch, barrier and max over ranks over gloo")
@@ -635,6 +667,20 @@ def secondary(torch, ea, device, stream, peaks, rank, barrier, max_over_ranks, w
             tb, _ = graph_time(torch, bstep, 50, stream, 3, barrier)
             out[name]["block_mask_build_us"] = 1e6 * tb / 50
             launches += 50
+    w = W.WORKLOADS[PRIMARY]
+    s = backward_setup(torch, ea, w, device, seed_shift=rank_seed_shift(rank))
+    bsteps = max(steps // 4, 10)
+    t, _ = graph_time(torch, s["step"], bsteps, stream, 5, barrier)
+    t = max_over_ranks(t)
+    ach = s["flops"] / (t / bsteps) / 1e12
+    out["backward_" + PRIMARY] = {
+        "value": weak_scaling_value(s["flops"] * bsteps, world, t) / 1e12, "unit": "TFLOP/s",
+        "ms_per_step": 1e3 * t / bsteps, "pairs": s["pairs"], "flops_per_step": s["flops"],
+        "flops_rule": "10*D*pairs (S, dP, dV, dK, dQ products)",
+        "roofline": {"bound": "tensor", "achieved": ach, "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                     "frac": ach / float(peaks["bf16_tflops"]), "traffic": None},
+        "kernels": "delta_kernel, attn_bwd_dkdv_kernel<128>, attn_bwd_dq_kernel<128>"}
+    launches += 3 * bsteps
     w = W.WORKLOADS["mqa_paged_decode_b32_kv32768"]
     s = decode_setup(torch, ea, w, device, seed_shift=rank_seed_shift(rank))
     t, _ = graph_time(torch, s["step"], steps, stream, 5, barrier)
@@ -660,6 +706,8 @@ def profile_arm(args):
         d = W.make_prefill_inputs(w)
         doc = torch.from_numpy(d["doc_id"]).to(device)
         step = lambda i: ea.attn_build_block_mask(w.S, w.S, doc_id=doc)  # noqa: E731
+    elif name.startswith("backward_"):
+        step = backward_setup(torch, ea, W.WORKLOADS[name[len("backward_"):]], device, 0)["step"]
     elif isinstance(W.WORKLOADS[name], W.Decode):
         step = decode_setup(torch, ea, W.WORKLOADS[name], device, 0)["step"]
     else:
