@@ -263,7 +263,7 @@ def backward_setup(torch, ea, w: W.Prefill, device, seed_shift: int):
         o, lse = ea.attn_fwd(q, k, v, **kw)
         sets.append((q, k, v, o, lse, do))
     dq, dk, dv = torch.empty_like(q0), torch.empty_like(k0), torch.empty_like(v0)
-    ws = torch.empty(ea.load_library().attn_bwd_workspace_bytes(w.B, w.Hq, w.S), dtype=torch.uint8, device=device)
+    ws = torch.empty(ea.attn_bwd_workspace_bytes(q0, k0, v0, **kw), dtype=torch.uint8, device=device)
     pairs = unmasked_pairs(w, d["doc_lens"])
 
     def step(i):

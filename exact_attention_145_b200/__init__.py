@@ -25,7 +25,7 @@ from ._lib import (ATTN_DEV_BAD_LEN, ATTN_DEV_BAD_MASK, ATTN_DEV_BAD_PAGE, ATTN_
                    MASK_DOCUMENT, MASK_NONE, MASK_WINDOW,
                    MOD_ALIBI, MOD_NONE, MOD_SOFTCAP, AttnError)
 
-__all__ = ["attn_fwd", "attn_bwd", "attn_decode", "attn_decode_noalloc", "attn_build_block_mask", "attn_lse_combine",
+__all__ = ["attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_decode", "attn_decode_noalloc", "attn_build_block_mask", "attn_lse_combine",
            "BlockMask", "AttnError",
            "load_library", "ATTN_DEV_TIMEOUT", "ATTN_DEV_BAD_PAGE", "ATTN_DEV_BAD_LEN",
            "ATTN_DEV_BAD_MASK"]
@@ -232,13 +232,8 @@ def attn_fwd(q, k, v, *, scale: Optional[float] = None, causal: bool = False, wi
     return out, lse
 
 
-def attn_bwd(q, k, v, out, lse, dout, *, scale: Optional[float] = None, causal: bool = False, window=None,
-             q_offset: int = 0, deterministic: bool = True, dq=None, dk=None, dv=None, workspace=None, status=None,
-             stream=None):
-    """Backward of attn_fwd: q [B, Sq, Hq, D], k/v [B, Skv, Hkv, D], the forward's
-    out (O) and lse [B, Hq, Sq], and the upstream gradient dout (shaped like q),
-    all bf16 except lse. Returns (dQ, dK, dV) shaped like q, k, v. Results are
-    deterministic whatever `deterministic` says."""
+def _bwd_params(q, k, v, out, lse, dout, dq, dk, dv, scale, causal, window, q_offset, deterministic, status):
+    """Checks the backward inputs and fills the C parameter block."""
     torch = _torch()
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
         _check_bf16(name, t, 4)
@@ -246,20 +241,15 @@ def attn_bwd(q, k, v, out, lse, dout, *, scale: Optional[float] = None, causal: 
     Skv, Hkv = k.shape[1], k.shape[2]
     if out.shape != q.shape or dout.shape != q.shape or v.shape != k.shape:
         raise ValueError("out and dout must be shaped like q, v like k")
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Sq) or not lse.is_contiguous():
+    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Sq) or not lse.is_contiguous()):
         raise ValueError("lse must be contiguous fp32 [B, Hq, Sq]")
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    lib = _lib.load()
-    if workspace is None:
-        workspace = torch.empty(max(lib.attn_bwd_workspace_bytes(B, Hq, Sq), 16), dtype=torch.uint8, device=q.device)
     p = _lib.BwdParams()
-    p.q, p.k, p.v, p.o, p.dout, p.lse = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
-                                         lse.data_ptr())
-    p.dq, p.dk, p.dv = dq.data_ptr(), dk.data_ptr(), dv.data_ptr()
+    p.q, p.k, p.v, p.o, p.dout = q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr()
+    p.lse = 0 if lse is None else lse.data_ptr()
+    p.dq, p.dk, p.dv = (0 if t is None else t.data_ptr() for t in (dq, dk, dv))
     for name, t in (("q_stride", q), ("k_stride", k), ("v_stride", v), ("o_stride", out), ("do_stride", dout),
-                    ("dq_stride", dq), ("dk_stride", dk), ("dv_stride", dv)):
+                    ("dq_stride", q if dq is None else dq), ("dk_stride", k if dk is None else dk),
+                    ("dv_stride", v if dv is None else dv)):
         setattr(p, name, _lib.c_i64x3(*t.stride()[:3]))
     p.B, p.Hq, p.Hkv, p.Sq, p.Skv, p.D = B, Hq, Hkv, Sq, Skv, D
     p.scale = 0.0 if scale is None else float(scale)
@@ -267,6 +257,36 @@ def attn_bwd(q, k, v, out, lse, dout, *, scale: Optional[float] = None, causal: 
     p.mask = spec
     p.deterministic = 1 if deterministic else 0
     p.status = _ptr(status)
+    return p
+
+
+def attn_bwd_workspace_bytes(q, k, v, *, causal: bool = False, window=None, q_offset: int = 0) -> int:
+    """Bytes of device workspace attn_bwd needs for these shapes and mask on
+    the current device (the delta rows, the dK/dV plan and the fp32 partials
+    of key tiles cut into pieces)."""
+    p = _bwd_params(q, k, v, q, None, q, None, None, None, None, causal, window, q_offset, True, None)
+    return int(_lib.load().attn_bwd_workspace_bytes(ctypes.byref(p)))
+
+
+def attn_bwd(q, k, v, out, lse, dout, *, scale: Optional[float] = None, causal: bool = False, window=None,
+             q_offset: int = 0, deterministic: bool = True, dq=None, dk=None, dv=None, workspace=None, status=None,
+             stream=None):
+    """Backward of attn_fwd: q [B, Sq, Hq, D], k/v [B, Skv, Hkv, D], the forward's
+    out (O) and lse [B, Hq, Sq], and the upstream gradient dout (shaped like q),
+    all bf16 except lse. Returns (dQ, dK, dV) shaped like q, k, v. Results are
+    deterministic whatever `deterministic` says. `workspace` (uint8, device)
+    needs attn_bwd_workspace_bytes(q, k, v, ...) bytes; allocated when None."""
+    torch = _torch()
+    if lse is None:
+        raise ValueError("lse is required")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    p = _bwd_params(q, k, v, out, lse, dout, dq, dk, dv, scale, causal, window, q_offset, deterministic, status)
+    lib = _lib.load()
+    if workspace is None:
+        workspace = torch.empty(max(int(lib.attn_bwd_workspace_bytes(ctypes.byref(p))), 16), dtype=torch.uint8,
+                                device=q.device)
     h = _stream_handle(q.device) if stream is None else stream
     _lib.check(lib.attn_bwd(ctypes.byref(p), workspace.data_ptr(), workspace.numel() * workspace.element_size(), h),
                "attn_bwd")

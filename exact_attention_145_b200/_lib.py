@@ -118,7 +118,7 @@ def load() -> ctypes.CDLL:
         lib.attn_decode.restype = ctypes.c_int
         lib.attn_decode_noalloc.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_void_p]
         lib.attn_decode_noalloc.restype = ctypes.c_int
-        lib.attn_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 3
+        lib.attn_bwd_workspace_bytes.argtypes = [ctypes.POINTER(BwdParams)]
         lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.attn_bwd.argtypes = [ctypes.POINTER(BwdParams), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
         lib.attn_bwd.restype = ctypes.c_int

@@ -195,22 +195,74 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (attn_status e = opt_in_smem(attn_bwd_dkdv_kernel<D>, L::kSmemBytes, r1, mu1)) return e;
   if (attn_status e = opt_in_smem(attn_bwd_dq_kernel<D>, L::kSmemBytes, r2, mu2)) return e;
   const int sms = sm_count();
-  a.n_units = a.B * a.Hkv * a.nK;
-  if (a.n_units > 0)
+  if (a.Skv > 0) {
+    a.n_units = a.B * a.Hkv * a.n_pieces;
     attn_bwd_dkdv_kernel<D><<<a.n_units < sms ? a.n_units : sms, kBwdThreads, L::kSmemBytes, st>>>(mq, mk, mv, mdo,
                                                                                                     a);
+    if (a.n_slots > 0)
+      attn_bwd_dkdv_reduce_kernel<D><<<dim3(a.nK, a.B * a.Hkv, kTile * D / kReduceElems), 256, 0, st>>>(a);
+  }
   a.n_units = a.B * a.Hq * a.nQ;
   attn_bwd_dq_kernel<D><<<a.n_units < sms ? a.n_units : sms, kBwdThreads, L::kSmemBytes, st>>>(mq, mk, mv, mdo, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// The dK/dV plan and workspace layout of a backward call: pieces per key
+// tile under a cap chosen so that there are about two pieces per SM (the
+// plan block on the device repeats the same integer arithmetic).
+struct BwdPlan {
+  int nQ, nK, g, mask, wl, wr, q_offset, cap, n_pieces, n_slots;
+  size_t off_pieces, off_tiles, off_part, bytes;
+};
+
+bool bwd_plan(const attn_bwd_params* p, int sms, BwdPlan* out) {
+  using namespace attn_bwd_kernels;
+  if (!p || p->B < 0 || p->Sq < 0 || p->Skv < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Hq % p->Hkv != 0) return false;
+  if (p->D != 64 && p->D != 128) return false;
+  if (p->mask.kind != ATTN_MASK_NONE && p->mask.kind != ATTN_MASK_CAUSAL && p->mask.kind != ATTN_MASK_WINDOW)
+    return false;
+  BwdPlan& q = *out;
+  q.g = p->Hq / p->Hkv;
+  q.mask = p->mask.kind;
+  q.q_offset = p->mask.kind == ATTN_MASK_NONE ? 0 : p->mask.q_offset;
+  q.wl = p->mask.kind == ATTN_MASK_WINDOW ? (p->mask.window_left < 0 ? -1 : p->mask.window_left) : -1;
+  q.wr = p->mask.kind == ATTN_MASK_CAUSAL
+             ? 0
+             : (p->mask.kind == ATTN_MASK_WINDOW ? (p->mask.window_right < 0 ? -1 : p->mask.window_right) : -1);
+  q.nQ = (p->Sq + kTile - 1) / kTile;
+  q.nK = (p->Skv + kTile - 1) / kTile;
+  long long total = 0;
+  int qlo;
+  for (int t = 0; t < q.nK; ++t)
+    total += kv_tile_steps(p->Sq, p->Skv, q.g, q.mask, q.wl, q.wr, q.q_offset, t, &qlo);
+  total *= (long long)p->B * p->Hkv;
+  const long long want = (total + 2LL * sms - 1) / (2LL * sms);
+  q.cap = (int)(want < 4 ? 4 : (want > (1LL << 30) ? (1LL << 30) : want));
+  long long np_sum = 0, slots = 0;
+  for (int t = 0; t < q.nK; ++t) {
+    const int np = kv_tile_pieces(kv_tile_steps(p->Sq, p->Skv, q.g, q.mask, q.wl, q.wr, q.q_offset, t, &qlo), q.cap);
+    np_sum += np;
+    slots += np > 1 ? np : 0;
+  }
+  if (np_sum * p->B * p->Hkv > 0x7fffffffLL || (long long)p->B * p->Hq * q.nQ > 0x7fffffffLL) return false;
+  q.n_pieces = (int)np_sum;
+  q.n_slots = (int)slots;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  q.off_pieces = up((size_t)p->B * p->Hq * p->Sq * sizeof(float));
+  q.off_tiles = q.off_pieces + up((size_t)q.n_pieces * 16);
+  q.off_part = q.off_tiles + up((size_t)(q.nK > 0 ? q.nK : 1) * 8);
+  q.bytes = q.off_part + (size_t)p->B * p->Hkv * q.n_slots * 2 * kTile * p->D * sizeof(float);
+  return true;
 }
 
 }  // namespace
 
 extern "C" {
 
-size_t attn_bwd_workspace_bytes(int B, int Hq, int Sq) {
-  if (B <= 0 || Hq <= 0 || Sq <= 0) return 0;
-  return ((size_t)B * Hq * Sq * sizeof(float) + 255) & ~size_t(255);
+size_t attn_bwd_workspace_bytes(const attn_bwd_params* p) {
+  BwdPlan plan;
+  if (!p || p->B <= 0 || p->Sq <= 0 || !bwd_plan(p, sm_count(), &plan)) return 0;
+  return plan.bytes;
 }
 
 attn_status attn_bwd(const attn_bwd_params* p, void* workspace, size_t workspace_bytes, void* stream) {
@@ -231,12 +283,51 @@ attn_status attn_bwd(const attn_bwd_params* p, void* workspace, size_t workspace
                               p->do_stride, p->dq_stride, p->dk_stride, p->dv_stride};
   for (const int64_t* st : strides)
     if (!strides_ok(st, 3)) return ATTN_ERR_UNSUPPORTED;
-  const size_t need = attn_bwd_workspace_bytes(p->B, p->Hq, p->Sq);
+  BwdPlan plan;
+  if (!bwd_plan(p, sm_count(), &plan)) return ATTN_ERR_UNSUPPORTED;
   if (!workspace || !aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
-  if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if (workspace_bytes < plan.bytes) return ATTN_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
 
-  // rowsum(dO o O) per (b, h, i)
+  BwdArgs a{};
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.Sq = p->Sq;
+  a.Skv = p->Skv;
+  a.g = plan.g;
+  a.scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
+  a.scale_log2 = a.scale * kLog2e;
+  a.mask = plan.mask;
+  a.q_offset = plan.q_offset;
+  a.wl = plan.wl;
+  a.wr = plan.wr;
+  a.nQ = plan.nQ;
+  a.nK = plan.nK;
+  a.lse = p->lse;
+  a.delta = reinterpret_cast<const float*>(ws);
+  a.dq = static_cast<__nv_bfloat16*>(p->dq);
+  a.dk = static_cast<__nv_bfloat16*>(p->dk);
+  a.dv = static_cast<__nv_bfloat16*>(p->dv);
+  a.dq_sb = p->dq_stride[0];
+  a.dq_ss = p->dq_stride[1];
+  a.dq_sh = p->dq_stride[2];
+  a.dk_sb = p->dk_stride[0];
+  a.dk_ss = p->dk_stride[1];
+  a.dk_sh = p->dk_stride[2];
+  a.dv_sb = p->dv_stride[0];
+  a.dv_ss = p->dv_stride[1];
+  a.dv_sh = p->dv_stride[2];
+  a.pieces = reinterpret_cast<const int4*>(ws + plan.off_pieces);
+  a.tiles = reinterpret_cast<const int2*>(ws + plan.off_tiles);
+  a.part = reinterpret_cast<float*>(ws + plan.off_part);
+  a.n_pieces = plan.n_pieces;
+  a.n_slots = plan.n_slots;
+  a.cap = plan.cap;
+  a.status = p->status;
+
+  // rowsum(dO o O) per (b, h, i); the extra last block writes the plan
   DeltaArgs da;
   da.o = static_cast<const __nv_bfloat16*>(p->o);
   da.dout = static_cast<const __nv_bfloat16*>(p->dout);
@@ -250,45 +341,13 @@ attn_status attn_bwd(const attn_bwd_params* p, void* workspace, size_t workspace
   da.Hq = p->Hq;
   da.Sq = p->Sq;
   da.D = p->D;
-  da.delta = static_cast<float*>(workspace);
+  da.delta = reinterpret_cast<float*>(ws);
   const int64_t rows = (int64_t)p->B * p->Hq * p->Sq;
-  if ((rows + 7) / 8 > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
-  delta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(da);
-
-  BwdArgs a{};
-  a.B = p->B;
-  a.Hq = p->Hq;
-  a.Hkv = p->Hkv;
-  a.Sq = p->Sq;
-  a.Skv = p->Skv;
-  a.g = p->Hq / p->Hkv;
-  a.scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->D));
-  a.scale_log2 = a.scale * kLog2e;
-  a.mask = p->mask.kind;
-  a.q_offset = p->mask.kind == ATTN_MASK_NONE ? 0 : p->mask.q_offset;
-  a.wl = p->mask.kind == ATTN_MASK_WINDOW ? (p->mask.window_left < 0 ? -1 : p->mask.window_left) : -1;
-  a.wr = p->mask.kind == ATTN_MASK_CAUSAL ? 0
-                                           : (p->mask.kind == ATTN_MASK_WINDOW
-                                                  ? (p->mask.window_right < 0 ? -1 : p->mask.window_right)
-                                                  : -1);
-  a.nQ = (p->Sq + kTile - 1) / kTile;
-  a.nK = (p->Skv + kTile - 1) / kTile;
-  a.lse = p->lse;
-  a.delta = static_cast<const float*>(workspace);
-  a.dq = static_cast<__nv_bfloat16*>(p->dq);
-  a.dk = static_cast<__nv_bfloat16*>(p->dk);
-  a.dv = static_cast<__nv_bfloat16*>(p->dv);
-  a.dq_sb = p->dq_stride[0];
-  a.dq_ss = p->dq_stride[1];
-  a.dq_sh = p->dq_stride[2];
-  a.dk_sb = p->dk_stride[0];
-  a.dk_ss = p->dk_stride[1];
-  a.dk_sh = p->dk_stride[2];
-  a.dv_sb = p->dv_stride[0];
-  a.dv_ss = p->dv_stride[1];
-  a.dv_sh = p->dv_stride[2];
-  a.status = p->status;
-  if ((long)a.B * a.Hq * a.nQ > 0x7fffffffL || (long)a.B * a.Hkv * a.nK > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+  const int rows_per_block = 256 / (p->D / 8);
+  const int64_t delta_blocks = (rows + rows_per_block - 1) / rows_per_block;
+  if (delta_blocks + 1 > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+  da.delta_blocks = (int)delta_blocks;
+  da.plan = a;
 
   CUtensorMap mq, mk, mv, mdo;
   const uint64_t dq[4] = {(uint64_t)p->D, (uint64_t)p->Sq, (uint64_t)p->Hq, (uint64_t)p->B};
@@ -305,6 +364,7 @@ attn_status attn_bwd(const attn_bwd_params* p, void* workspace, size_t workspace
   // With Skv == 0 no key tile is ever loaded; the unused maps point at Q.
   if (attn_status e = make_map(&mk, p->Skv > 0 ? p->k : p->q, 4, p->Skv > 0 ? dk : dq, sk, kTile, 1)) return e;
   if (attn_status e = make_map(&mv, p->Skv > 0 ? p->v : p->q, 4, p->Skv > 0 ? dk : dq, sv, kTile, 1)) return e;
+  delta_kernel<<<(unsigned)(delta_blocks + 1), kPlanThreads, 0, st>>>(da);
   return p->D == 128 ? launch_bwd<128>(mq, mk, mv, mdo, a, st) : launch_bwd<64>(mq, mk, mv, mdo, a, st);
 }
 

@@ -2,24 +2,31 @@
 // O = softmax(scale * Q K^T + mask) V for an upstream gradient dO, with the
 // forward's log-sum-exp as input. The FlashAttention overview ("Examples")
 // names this backward pass and its deterministic option; the kernels here
-// are deterministic by construction: every output element is accumulated by
-// one CTA in a fixed order, with no atomics.
+// are deterministic by construction: every output element is accumulated in
+// a fixed order, with no atomics.
 //
 // With P = exp(scale * S - LSE) (S = Q K^T, masked entries 0), the chain rule
 // gives dV = P^T dO, dP = dO V^T, dS = P o (dP - delta) with delta_i =
-// dO_i . O_i, dQ = scale * dS K and dK = scale * dS^T Q. Three kernels:
-//   delta_kernel   delta_i for every (b, h, i) on CUDA cores;
-//   dkdv kernel    one work unit per (b, KV head, 128-key tile): loops over
-//                  every query tile and every query head of the group,
-//                  recomputing S^T = K Q^T and dP^T = V dO^T in TMEM, writing
-//                  P^T and dS^T back to TMEM as bf16 and accumulating
-//                  dV += P^T dO and dK += dS^T Q there (tcgen05, A from TMEM);
+// dO_i . O_i, dQ = scale * dS K and dK = scale * dS^T Q. Four kernels:
+//   delta_kernel   delta_i for every (b, h, i) on CUDA cores; its last block
+//                  writes the dK/dV work plan (below);
+//   dkdv kernel    one work unit per piece of a (b, KV head, 128-key tile):
+//                  a contiguous range of the tile's steps (query tile x query
+//                  head of the group), recomputing S^T = K Q^T and
+//                  dP^T = V dO^T in TMEM, writing P^T and dS^T back to TMEM
+//                  as bf16 and accumulating dV += P^T dO and dK += dS^T Q
+//                  there (tcgen05, A from TMEM);
+//   dkdv reduce    sums the fp32 partials of key tiles cut into several
+//                  pieces, in piece order;
 //   dq kernel      one work unit per (b, query head, 128-row tile): loops over
 //                  the key tiles, S = Q K^T and dP = dO V^T in TMEM, dS back
 //                  to TMEM as bf16, dQ += dS K.
-// Warp roles (256 threads): warps 0-3 compute (thread = TMEM lane = key row
-// in dkdv, query row in dq), warp 4 MMA issue (owns TMEM), warp 5 TMA
-// producer, warps 6-7 idle. Every wait is bounded (sm100.cuh).
+// Pieces balance the causal triangle: key tile 0 meets every query tile,
+// the last key tile one, so whole tiles as units would leave the first
+// CTAs with several times the mean work.
+// Warp roles (320 threads): warps 0-7 compute (warp w: TMEM lanes
+// 32 (w % 4) .. +31 = the tile's rows, columns half w / 4), warp 8 MMA issue
+// (owns TMEM), warp 9 TMA producer. Every wait is bounded (sm100.cuh).
 #pragma once
 
 #include <cstdint>
@@ -33,12 +40,40 @@ namespace attn_bwd_kernels {
 using namespace attn_sm100;
 
 constexpr int kTile = 128;  // rows of a Q tile, keys of a K/V tile
-constexpr int kBwdThreads = 256;
-constexpr int kBMmaWarp = 4;
-constexpr int kBTmaWarp = 5;
+constexpr int kBwdThreads = 320;
+constexpr int kBCompute = 256;  // compute threads: two per tile row
+constexpr int kBMmaWarp = 8;
+constexpr int kBTmaWarp = 9;
+constexpr int kPlanThreads = 256;
 constexpr float kLog2eB = 1.4426950408889634f;
 enum : int { BMASK_NONE = 0, BMASK_CAUSAL = 1, BMASK_WINDOW = 2 };
 enum : int { BDEV_TIMEOUT = 1 };
+
+// Steps of key tile t in the dK/dV pass: (query tiles that meet it) x g.
+// *qlo receives the first such query tile. Shared by the host (workspace
+// sizing, grid) and the plan block, so both count the same pieces.
+__host__ __device__ inline int kv_tile_steps(int Sq, int Skv, int g, int mask, int wl, int wr, int q_offset, int t,
+                                             int* qlo) {
+  const long long k0 = (long long)t * kTile;
+  const long long kend = (long long)(t + 1) * kTile < (long long)Skv ? (long long)(t + 1) * kTile : (long long)Skv;
+  const long long k1 = kend - 1;
+  long long lo = 0, hi = (long long)Sq - 1;
+  if (mask != BMASK_NONE) {
+    // key k is seen by q_pos in [k - wr, k + wl]; q_pos = i + q_offset
+    if (wr >= 0 && k0 - wr - q_offset > lo) lo = k0 - wr - q_offset;
+    if (wl >= 0 && k1 + wl - q_offset < hi) hi = k1 + wl - q_offset;
+  }
+  if (hi < lo) {
+    *qlo = 0;
+    return 0;
+  }
+  *qlo = (int)(lo / kTile);
+  return (int)(hi / kTile - lo / kTile + 1) * g;
+}
+
+// Pieces of a key tile with n steps under a piece cap: at least one (a tile
+// no query sees still writes its zero gradients).
+__host__ __device__ inline int kv_tile_pieces(int n, int cap) { return n <= cap ? 1 : (n + cap - 1) / cap; }
 
 struct BwdArgs {
   int B, Hq, Hkv, Sq, Skv, g;
@@ -49,57 +84,117 @@ struct BwdArgs {
   const float* delta;  // [B][Hq][Sq] (workspace, written by delta_kernel)
   __nv_bfloat16 *dq, *dk, *dv;
   int64_t dq_sb, dq_ss, dq_sh, dk_sb, dk_ss, dk_sh, dv_sb, dv_ss, dv_sh;
+  // dK/dV plan (workspace, written by the delta kernel's last block):
+  const int4* pieces;  // [n_pieces] {key tile, first step, end step, partial slot or -1}
+  const int2* tiles;   // [nK] {pieces of the tile, first partial slot or -1}
+  float* part;         // [B * Hkv][n_slots][2][128][D] fp32 partial dV, dK (dK without the scale)
+  int n_pieces, n_slots, cap;
   int n_units;
   int* status;
 };
 
-// ---------------------------------------------------------------- delta
-// delta[b][h][i] = sum_d dO[b,i,h,d] * O[b,i,h,d]; one warp per row.
+// ---------------------------------------------------------------- delta + plan
+// delta[b][h][i] = sum_d dO[b,i,h,d] * O[b,i,h,d]; D / 8 threads per row,
+// 16-byte loads. The last block writes the dK/dV plan instead.
 struct DeltaArgs {
   const __nv_bfloat16 *o, *dout;
   int64_t o_sb, o_ss, o_sh, do_sb, do_ss, do_sh;
   int B, Hq, Sq, D;
   float* delta;
+  int delta_blocks;
+  BwdArgs plan;  // mask and sizes for the plan; pieces / tiles written through const_cast
 };
 
-__global__ void __launch_bounds__(256) delta_kernel(const DeltaArgs a) {
-  const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
-  const int lane = threadIdx.x % 32;
-  if (row >= (int64_t)a.B * a.Hq * a.Sq) return;
-  const int i = (int)(row % a.Sq);
-  const int h = (int)((row / a.Sq) % a.Hq);
-  const int b = (int)(row / ((int64_t)a.Sq * a.Hq));
-  const __nv_bfloat16* o = a.o + b * a.o_sb + (int64_t)i * a.o_ss + (int64_t)h * a.o_sh;
-  const __nv_bfloat16* d = a.dout + b * a.do_sb + (int64_t)i * a.do_ss + (int64_t)h * a.do_sh;
+__device__ __forceinline__ float dot8_bf16(uint4 x, uint4 y) {
+  const __nv_bfloat162* a = reinterpret_cast<const __nv_bfloat162*>(&x);
+  const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&y);
   float acc = 0.f;
-  for (int c = 2 * lane; c < a.D; c += 64) {
-    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + c));
-    const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(d + c));
-    acc = fmaf(x.x, y.x, acc);
-    acc = fmaf(x.y, y.y, acc);
-  }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) a.delta[((int64_t)b * a.Hq + h) * a.Sq + i] = acc;
+  for (int i = 0; i < 4; ++i) {
+    const float2 u = __bfloat1622float2(a[i]), v = __bfloat1622float2(b[i]);
+    acc = fmaf(u.x, v.x, acc);
+    acc = fmaf(u.y, v.y, acc);
+  }
+  return acc;
+}
+
+// Block-wide exclusive scan of two counters (kPlanThreads threads).
+__device__ __forceinline__ void block_scan2(int& a, int& b, int* sh) {
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  int ia = a, ib = b;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int ya = __shfl_up_sync(0xffffffffu, ia, off), yb = __shfl_up_sync(0xffffffffu, ib, off);
+    if (lane >= off) {
+      ia += ya;
+      ib += yb;
+    }
+  }
+  if (lane == 31) {
+    sh[warp] = ia;
+    sh[32 + warp] = ib;
+  }
+  __syncthreads();
+  int ba = 0, bb = 0;
+  for (int w = 0; w < warp; ++w) {
+    ba += sh[w];
+    bb += sh[32 + w];
+  }
+  a = ba + ia - a;
+  b = bb + ib - b;
+}
+
+__device__ void write_plan(const BwdArgs& p) {
+  __shared__ int sh[64];
+  const int nK = p.nK;
+  const int per = (nK + kPlanThreads - 1) / kPlanThreads;
+  const int t0 = min((int)threadIdx.x * per, nK), t1 = min(t0 + per, nK);
+  int np_sum = 0, slot_sum = 0, qlo;
+  for (int t = t0; t < t1; ++t) {
+    const int np = kv_tile_pieces(kv_tile_steps(p.Sq, p.Skv, p.g, p.mask, p.wl, p.wr, p.q_offset, t, &qlo), p.cap);
+    np_sum += np;
+    slot_sum += np > 1 ? np : 0;
+  }
+  int ps = np_sum, ss = slot_sum;
+  block_scan2(ps, ss, sh);
+  int4* pieces = const_cast<int4*>(p.pieces);
+  int2* tiles = const_cast<int2*>(p.tiles);
+  for (int t = t0; t < t1; ++t) {
+    const int n = kv_tile_steps(p.Sq, p.Skv, p.g, p.mask, p.wl, p.wr, p.q_offset, t, &qlo);
+    const int np = kv_tile_pieces(n, p.cap);
+    tiles[t] = make_int2(np, np > 1 ? ss : -1);
+    for (int j = 0; j < np; ++j)
+      pieces[ps + j] = make_int4(t, (int)((long long)j * n / np), (int)((long long)(j + 1) * n / np), np > 1 ? ss + j : -1);
+    ps += np;
+    ss += np > 1 ? np : 0;
+  }
+}
+
+__global__ void __launch_bounds__(256) delta_kernel(const DeltaArgs a) {
+  if ((int)blockIdx.x == a.delta_blocks) {
+    write_plan(a.plan);
+    return;
+  }
+  const int tpr = a.D / 8;  // threads per row
+  const int rows_per_block = 256 / tpr;
+  const int64_t row = (int64_t)blockIdx.x * rows_per_block + threadIdx.x / tpr;
+  const int part = threadIdx.x % tpr;
+  const bool live = row < (int64_t)a.B * a.Hq * a.Sq;
+  float acc = 0.f;
+  int i = 0, h = 0, b = 0;
+  if (live) {
+    i = (int)(row % a.Sq);
+    h = (int)((row / a.Sq) % a.Hq);
+    b = (int)(row / ((int64_t)a.Sq * a.Hq));
+    const __nv_bfloat16* o = a.o + b * a.o_sb + (int64_t)i * a.o_ss + (int64_t)h * a.o_sh + part * 8;
+    const __nv_bfloat16* d = a.dout + b * a.do_sb + (int64_t)i * a.do_ss + (int64_t)h * a.do_sh + part * 8;
+    acc = dot8_bf16(*reinterpret_cast<const uint4*>(o), *reinterpret_cast<const uint4*>(d));
+  }
+  for (int off = tpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (live && part == 0) a.delta[((int64_t)b * a.Hq + h) * a.Sq + i] = acc;
 }
 
 // ---------------------------------------------------------------- masks
-// Query tiles [lo, hi] that meet key tile t (keys k0..k1) under the window
-// form; false when none.
-__device__ __forceinline__ bool q_range_for_k(const BwdArgs& a, int t, int& lo, int& hi) {
-  const long k0 = (long)t * kTile, k1 = min((long)(t + 1) * kTile, (long)a.Skv) - 1;
-  long qlo = 0, qhi = (long)a.Sq - 1;
-  if (a.mask != BMASK_NONE) {
-    // key k is seen by q_pos in [k - wr, k + wl]; q_pos = i + q_offset
-    if (a.wr >= 0) qlo = max(qlo, k0 - a.wr - a.q_offset);
-    if (a.wl >= 0) qhi = min(qhi, k1 + a.wl - a.q_offset);
-  }
-  if (qhi < qlo) return false;
-  lo = (int)(qlo / kTile);
-  hi = (int)(qhi / kTile);
-  return true;
-}
-
 // Key tiles [lo, hi] that meet query tile qt.
 __device__ __forceinline__ bool k_range_for_q(const BwdArgs& a, int qt, int& lo, int& hi) {
   const long q0 = (long)qt * kTile + a.q_offset, q1 = min((long)(qt + 1) * kTile, (long)a.Sq) - 1 + a.q_offset;
@@ -142,11 +237,11 @@ template <int D>
 struct BLayout {
   static constexpr int kTileBytes = kTile * D * 2;    // one operand tile (128 rows x D bf16)
   static constexpr int kChunk = kTile * 64 * 2;       // one 128-row x 64-column SW128 box
-  // dkdv: K, V of the unit, then a 2-slot ring of (Q, dO, lse, delta) per step.
+  // dkdv: K, V of the unit, then a 2-slot ring of (Q, dO) per step.
   // dq: Q, dO of the unit, then a 2-slot ring of (K, V) per step.
   static constexpr int kFixOff = 0;                   // two unit tiles
   static constexpr int kRingOff = 2 * kTileBytes;     // 2 slots x two step tiles
-  static constexpr int kVecOff = kRingOff + 4 * kTileBytes;  // dkdv: 2 slots x (lse, delta) x 128 floats
+  static constexpr int kVecOff = kRingOff + 4 * kTileBytes;  // dkdv: 2 slots x (log2e*LSE, delta) x 128 floats
   static constexpr int kBarOff = kVecOff + 2 * 2 * kTile * 4;
   // Each CTA allocates all 512 TMEM columns, so two CTAs must never share an
   // SM: the request is padded past half of the SM's 228 KB of shared memory.
@@ -160,31 +255,40 @@ struct BBarriers {
   uint64_t fix_full, fix_empty;  // unit tiles loaded / released
   uint64_t ring_full[2], ring_empty[2];
   uint64_t mm1_ready;   // the step's first two products (S / dP) are in TMEM
-  uint64_t comp_ready;  // the compute warps wrote P^T / dS^T (dkdv) or dS (dq): 128 arrivals
+  uint64_t comp_ready;  // the compute warps wrote P^T / dS^T (dkdv) or dS (dq): 256 arrivals
   uint64_t acc_done;    // the unit's accumulators are final
-  uint64_t acc_free;    // the epilogue read them: 128 arrivals
-  uint64_t vec_ready[2];  // dkdv: the step's LSE / delta columns are in shared memory (128 arrivals)
+  uint64_t acc_free;    // the epilogue read them: 256 arrivals
+  uint64_t vec_ready[2];  // dkdv: the step's LSE / delta columns are in shared memory (256 arrivals)
   uint64_t final_mma;
   uint32_t tmem_base;
   int abort_flag;
 };
 
+// The bf16 result of 32-column chunk c (P^T / dS^T / dS) is packed into the
+// first 16 columns of the chunk's own source columns, so that the two
+// column halves of a tile never write where the other half still reads.
+// A-operand column of the TS MMA over rows 16 kk .. 16 kk + 15 of the
+// contraction:
+__device__ __forceinline__ uint32_t packed_col(int kk) { return 32u * (uint32_t)(kk >> 1) + 8u * (uint32_t)(kk & 1); }
+
 // ---------------------------------------------------------------- work maps
-// dkdv unit u -> (b, hk, key tile t); t ascending is heaviest first for the
-// causal form. Steps: q tiles qt of [lo, hi] times the g query heads.
+// dkdv unit u -> piece pid = u / (B * Hkv) of group (b, hk) = u % (B * Hkv).
+// Pieces are numbered by key tile, so the causal heavy tiles come first.
 struct KvUnit {
-  int b, hk, t, qlo, n;  // n = steps
+  int b, hk, t, qlo, s0, n, slot;  // steps s0 .. s0 + n - 1; slot >= 0: write fp32 partials
 };
 __device__ __forceinline__ KvUnit kv_unit(const BwdArgs& a, int u) {
   KvUnit w;
   const int per = a.B * a.Hkv;
-  w.t = u / per;
-  const int r = u % per;
-  w.b = r / a.Hkv;
-  w.hk = r % a.Hkv;
-  int lo = 0, hi = -1;
-  w.n = q_range_for_k(a, w.t, lo, hi) ? (hi - lo + 1) * a.g : 0;
-  w.qlo = lo;
+  const int pid = u / per, grp = u % per;
+  w.b = grp / a.Hkv;
+  w.hk = grp % a.Hkv;
+  const int4 pc = a.pieces[pid];
+  w.t = pc.x;
+  w.s0 = pc.y;
+  w.n = pc.z - pc.y;
+  w.slot = pc.w;
+  kv_tile_steps(a.Sq, a.Skv, a.g, a.mask, a.wl, a.wr, a.q_offset, w.t, &w.qlo);
   return w;
 }
 // dq unit u -> (b, h, q tile qt); last q tiles first (the most key tiles).
@@ -212,7 +316,6 @@ __device__ __forceinline__ float bex2(float x) {
 
 // ---------------------------------------------------------------- dK / dV
 // TMEM columns: S^T [0, 128), dP^T [128, 256), dV [256, 256 + D), dK [256 + D, 256 + 2D).
-// P^T (bf16 pairs) replaces the first 64 columns of S^T, dS^T the first 64 of dP^T.
 // MMA order per step: S^T, dP^T | (compute) | dV, dK, S^T(next), dP^T(next).
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -234,11 +337,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bar.ring_empty[i], 1);
     }
     mbar_init(&bar.mm1_ready, 1);
-    mbar_init(&bar.comp_ready, kTile);
+    mbar_init(&bar.comp_ready, kBCompute);
     mbar_init(&bar.acc_done, 1);
-    mbar_init(&bar.acc_free, kTile);
-    mbar_init(&bar.vec_ready[0], kTile);
-    mbar_init(&bar.vec_ready[1], kTile);
+    mbar_init(&bar.acc_free, kBCompute);
+    mbar_init(&bar.vec_ready[0], kBCompute);
+    mbar_init(&bar.vec_ready[1], kBCompute);
     mbar_init(&bar.final_mma, 1);
     fence_barrier_init();
   }
@@ -287,7 +390,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       __syncwarp();
       ++ucnt;
-      for (int s = 0; s < w.n; ++s, ++gstep) {
+      for (int s = w.s0; s < w.s0 + w.n; ++s, ++gstep) {
         const int slot = gstep & 1, use = gstep >> 1;
         if (use > 0 && !wait_all(&bar.ring_empty[slot], (use - 1) & 1)) { ok = false; break; }
         const int qt = w.qlo + s / a.g, h = w.hk * a.g + s % a.g;
@@ -355,16 +458,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         if (elect_one_sync()) {
           const uint32_t qmn = ring_mn + (uint32_t)slot * 2 * kTileUnits, dmn = qmn + kTileUnits;
-          // dV += P^T dO: P^T from TMEM columns [0, 64), dO rows 16kk..
+          // dV += P^T dO: P^T packed in S^T's columns, dO rows 16kk..
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + 256, tmem + kk * 8, sdesc_join(dmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
+            mma_ts(tmem + 256, tmem + packed_col(kk), sdesc_join(dmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
                    (s > 0 || kk > 0) ? 1u : 0u);
-          // dK += dS^T Q: dS^T from TMEM columns [128, 192)
+          // dK += dS^T Q: dS^T packed in dP^T's columns
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + 256 + D, tmem + 128 + kk * 8, sdesc_join(qmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
-                   (s > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + 256 + D, tmem + 128 + packed_col(kk), sdesc_join(qmn + ((kk * 16 * 128) >> 4), kHi),
+                   idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bar.ring_empty[slot]);
           if (!more) {
             mma_commit(&bar.acc_done);
@@ -381,62 +484,72 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (elect_one_sync()) mma_commit(&bar.final_mma);
     __syncwarp();
     mbar_wait_timeout(&bar.final_mma, 0);
-  } else if (warp < 4) {
+  } else {
     // ------------------------------------------------------------ compute
-    const int row = threadIdx.x;  // key row of the tile = TMEM lane
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int row = threadIdx.x % kTile;  // key row of the tile = TMEM lane
+    const int half = warp / 4;            // columns [64 half, 64 half + 64) of S^T / dP^T
+    const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     int ucnt = 0, gstep = 0;
     bool ok = true;
     const float NEG_INF = -__int_as_float(0x7f800000);
+    const float POS_INF = __int_as_float(0x7f800000);
     for (int r = 0; ok && r < rounds; ++r) {
       const int u = unit_of(r);
       if (u < 0) continue;
       const KvUnit w = kv_unit(a, u);
       const long key = (long)w.t * kTile + row;
+      const bool real = key < a.Skv;
+      const int c_lo = half * (D / 2);  // this thread's output columns [c_lo, c_lo + D / 2)
       if (w.n == 0) {
         // no query sees these keys: their gradients are exactly zero
-        if (key < a.Skv) {
-          __nv_bfloat16* dvr = a.dv + w.b * a.dv_sb + key * a.dv_ss + (int64_t)w.hk * a.dv_sh;
-          __nv_bfloat16* dkr = a.dk + w.b * a.dk_sb + key * a.dk_ss + (int64_t)w.hk * a.dk_sh;
-          for (int c = 0; c < D; c += 8) {
+        if (real) {
+          __nv_bfloat16* dvr = a.dv + w.b * a.dv_sb + key * a.dv_ss + (int64_t)w.hk * a.dv_sh + c_lo;
+          __nv_bfloat16* dkr = a.dk + w.b * a.dk_sb + key * a.dk_ss + (int64_t)w.hk * a.dk_sh + c_lo;
+          for (int c = 0; c < D / 2; c += 8) {
             *reinterpret_cast<uint4*>(dvr + c) = make_uint4(0, 0, 0, 0);
             *reinterpret_cast<uint4*>(dkr + c) = make_uint4(0, 0, 0, 0);
           }
         }
         continue;
       }
+      // queries that see this key: q_pos in [key - wr, key + wl], q_pos = i + q_offset
+      long qlo_i = 0, qhi_i = (long)a.Sq - 1;
+      if (a.mask != BMASK_NONE) {
+        if (a.wr >= 0) qlo_i = max(qlo_i, key - a.wr - a.q_offset);
+        if (a.wl >= 0) qhi_i = min(qhi_i, key + a.wl - a.q_offset);
+      }
+      if (!real) qhi_i = -1;
       for (int s = 0; s < w.n; ++s) {
         const int g = gstep + s, slot = g & 1;
-        const int qt = w.qlo + s / a.g, h = w.hk * a.g + s % a.g;
-        // Column values of the step (LSE and delta of the q tile's queries):
-        // thread r fetches query qt*128 + r into a shared, double-buffered
-        // array; a bounded mbarrier (128 arrivals) publishes it.
+        const int qt = w.qlo + (w.s0 + s) / a.g, h = w.hk * a.g + (w.s0 + s) % a.g;
+        // Column values of the step (log2e * LSE and delta of the q tile's
+        // queries): half 0 fetches the LSE of query qt*128 + row, half 1 its
+        // delta, into a shared, double-buffered array; a bounded mbarrier
+        // (256 arrivals) publishes it.
         float* vec = reinterpret_cast<float*>(smem + L::kVecOff) + slot * 2 * kTile;
         {
           const int qi = qt * kTile + row;
-          float lv = NEG_INF, dv = 0.f;
+          float val = half == 0 ? POS_INF : 0.f;
           if (qi < a.Sq) {
             const int64_t ix = ((int64_t)w.b * a.Hq + h) * a.Sq + qi;
-            lv = a.lse[ix];
-            dv = a.delta[ix];
+            if (half == 0) {
+              const float l = a.lse[ix];
+              // LSE -inf (a row with no allowed key): none of its pairs is allowed either
+              val = l == NEG_INF ? POS_INF : l * kLog2eB;
+            } else {
+              val = a.delta[ix];
+            }
           }
-          vec[row] = lv;
-          vec[kTile + row] = dv;
+          vec[half * kTile + row] = val;
           mbar_arrive(&bar.vec_ready[slot]);
         }
         if (!wait_spin_all(&bar.mm1_ready, g & 1)) { ok = false; break; }
         if (!wait_spin_all(&bar.vec_ready[slot], (g >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const bool full = pair_full(a, qt, w.t);
-        // queries that see this key: q_pos in [key - wr, key + wl], q_pos = i + q_offset
-        long qlo_i = 0, qhi_i = (long)a.Sq - 1;
-        if (a.mask != BMASK_NONE) {
-          if (a.wr >= 0) qlo_i = max(qlo_i, key - a.wr - a.q_offset);
-          if (a.wl >= 0) qhi_i = min(qhi_i, key + a.wl - a.q_offset);
-        }
-        if (key >= a.Skv) qhi_i = -1;
 #pragma unroll 1
-        for (int c = 0; c < kTile / 32; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * half + cc;
           float x[32], dp[32];
           tmem_ld32f(lane_base + 32 * c, x);
           tmem_ld32f(lane_base + 128 + 32 * c, dp);
@@ -444,63 +557,82 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           reg_fence_f<32>(x);
           reg_fence_f<32>(dp);
           const uint32_t bits = full ? 0xffffffffu : range_bits(qlo_i, qhi_i, (long)qt * kTile + 32 * c);
+          const float4* l2v = reinterpret_cast<const float4*>(vec + 32 * c);
+          const float4* dlv = reinterpret_cast<const float4*>(vec + kTile + 32 * c);
           uint32_t pk[16], dk[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pe[2], de[2];
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 l4 = l2v[e4], d4 = dlv[e4];
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pe[4], de[4];
 #pragma unroll
-            for (int z = 0; z < 2; ++z) {
-              const int col = 32 * c + e + z;
-              // LSE -inf (a row with no allowed key): no pair of it is allowed either
-              const float l2 = vec[col] == NEG_INF ? __int_as_float(0x7f800000) : vec[col] * kLog2eB;
-              const bool on = (bits >> (e + z)) & 1u;
-              const float p = on ? bex2(fmaf(x[e + z], a.scale_log2, -l2)) : 0.f;
+            for (int z = 0; z < 4; ++z) {
+              const int e = 4 * e4 + z;
+              const float p = ((bits >> e) & 1u) ? bex2(fmaf(x[e], a.scale_log2, -lv[z])) : 0.f;
               pe[z] = p;
-              de[z] = p * (dp[e + z] - vec[kTile + col]);
+              de[z] = p * (dp[e] - dv[z]);
             }
-            pk[e / 2] = pack_bf16x2(pe[0], pe[1]);
-            dk[e / 2] = pack_bf16x2(de[0], de[1]);
+            pk[2 * e4] = pack_bf16x2(pe[0], pe[1]);
+            pk[2 * e4 + 1] = pack_bf16x2(pe[2], pe[3]);
+            dk[2 * e4] = pack_bf16x2(de[0], de[1]);
+            dk[2 * e4 + 1] = pack_bf16x2(de[2], de[3]);
           }
-          // P^T chunk c -> columns [16c, 16c + 16) (S^T columns already read),
-          // dS^T chunk c -> [128 + 16c, 128 + 16c + 16) likewise
-          tmem_st16(lane_base + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(pk));
-          tmem_st16(lane_base + 128 + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(dk));
+          // P^T and dS^T of chunk c -> the first 16 of its own 32 source columns
+          tmem_st16(lane_base + 32 * c, *reinterpret_cast<uint32_t(*)[16]>(pk));
+          tmem_st16(lane_base + 128 + 32 * c, *reinterpret_cast<uint32_t(*)[16]>(dk));
         }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bar.comp_ready);
       }
       if (!ok) break;
-      // epilogue: dV, dK (x scale) rows -> bf16
+      // epilogue: dV, dK rows, this thread's half of the columns
       if (!wait_all(&bar.acc_done, ucnt & 1)) break;
       tc_fence_after();
       {
         // tcgen05.ld is warp-collective: every lane loads, only rows of real
         // keys are stored (a ragged tile splits a warp).
-        const bool real = key < a.Skv;
-        __nv_bfloat16* dvr = a.dv + w.b * a.dv_sb + (real ? key : 0) * a.dv_ss + (int64_t)w.hk * a.dv_sh;
-        __nv_bfloat16* dkr = a.dk + w.b * a.dk_sb + (real ? key : 0) * a.dk_ss + (int64_t)w.hk * a.dk_sh;
+        const long krow = real ? key : 0;
+        __nv_bfloat16* dvr = a.dv + w.b * a.dv_sb + krow * a.dv_ss + (int64_t)w.hk * a.dv_sh + c_lo;
+        __nv_bfloat16* dkr = a.dk + w.b * a.dk_sb + krow * a.dk_ss + (int64_t)w.hk * a.dk_sh + c_lo;
+        float* pv = nullptr;
+        float* pkp = nullptr;
+        if (w.slot >= 0) {
+          const int grp = w.b * a.Hkv + w.hk;
+          float* base = a.part + ((size_t)grp * a.n_slots + w.slot) * 2 * kTile * D;
+          pv = base + (size_t)row * D + c_lo;
+          pkp = base + (size_t)kTile * D + (size_t)row * D + c_lo;
+        }
 #pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
+        for (int c = 0; c < D / 2; c += 32) {
           float v0[32], k0[32];
-          tmem_ld32f(lane_base + 256 + c, v0);
-          tmem_ld32f(lane_base + 256 + D + c, k0);
+          tmem_ld32f(lane_base + 256 + c_lo + c, v0);
+          tmem_ld32f(lane_base + 256 + D + c_lo + c, k0);
           tmem_ld_wait();
           reg_fence_f<32>(v0);
           reg_fence_f<32>(k0);
+          if (w.slot >= 0) {
+            // partial of a split key tile: fp32, every row (the reduction skips ragged rows)
 #pragma unroll
-          for (int e = 0; real && e < 32; e += 8) {
-            uint4 pv, pkk;
-            pv.x = pack_bf16x2(v0[e], v0[e + 1]);
-            pv.y = pack_bf16x2(v0[e + 2], v0[e + 3]);
-            pv.z = pack_bf16x2(v0[e + 4], v0[e + 5]);
-            pv.w = pack_bf16x2(v0[e + 6], v0[e + 7]);
-            pkk.x = pack_bf16x2(k0[e] * a.scale, k0[e + 1] * a.scale);
-            pkk.y = pack_bf16x2(k0[e + 2] * a.scale, k0[e + 3] * a.scale);
-            pkk.z = pack_bf16x2(k0[e + 4] * a.scale, k0[e + 5] * a.scale);
-            pkk.w = pack_bf16x2(k0[e + 6] * a.scale, k0[e + 7] * a.scale);
-            *reinterpret_cast<uint4*>(dvr + c + e) = pv;
-            *reinterpret_cast<uint4*>(dkr + c + e) = pkk;
+            for (int e = 0; e < 32; e += 4) {
+              *reinterpret_cast<float4*>(pv + c + e) = make_float4(v0[e], v0[e + 1], v0[e + 2], v0[e + 3]);
+              *reinterpret_cast<float4*>(pkp + c + e) = make_float4(k0[e], k0[e + 1], k0[e + 2], k0[e + 3]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; real && e < 32; e += 8) {
+              uint4 pvv, pkk;
+              pvv.x = pack_bf16x2(v0[e], v0[e + 1]);
+              pvv.y = pack_bf16x2(v0[e + 2], v0[e + 3]);
+              pvv.z = pack_bf16x2(v0[e + 4], v0[e + 5]);
+              pvv.w = pack_bf16x2(v0[e + 6], v0[e + 7]);
+              pkk.x = pack_bf16x2(k0[e] * a.scale, k0[e + 1] * a.scale);
+              pkk.y = pack_bf16x2(k0[e + 2] * a.scale, k0[e + 3] * a.scale);
+              pkk.z = pack_bf16x2(k0[e + 4] * a.scale, k0[e + 5] * a.scale);
+              pkk.w = pack_bf16x2(k0[e + 6] * a.scale, k0[e + 7] * a.scale);
+              *reinterpret_cast<uint4*>(dvr + c + e) = pvv;
+              *reinterpret_cast<uint4*>(dkr + c + e) = pkk;
+            }
           }
           __syncwarp();  // reconverge before the next warp-collective load
         }
@@ -521,9 +653,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0 && bar.abort_flag && a.status) atomicOr(a.status, BDEV_TIMEOUT);
 }
 
+// Sums the partials of key tiles that were cut into several pieces, in piece
+// order, and writes dV and scale * dK as bf16. Grid (nK, B * Hkv,
+// 128 * D / 1024): each block sums 1024 consecutive elements (1024 / D rows)
+// of both tiles, one float4 per thread.
+constexpr int kReduceElems = 1024;
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_dkdv_reduce_kernel(const BwdArgs a) {
+  const int t = blockIdx.x, grp = blockIdx.y;
+  const int2 tl = a.tiles[t];
+  if (tl.x <= 1) return;
+  const int b = grp / a.Hkv, hk = grp % a.Hkv;
+  const size_t tile_elems = (size_t)kTile * D;
+  const float* base = a.part + ((size_t)grp * a.n_slots + tl.y) * 2 * tile_elems;
+  const int idx = blockIdx.z * kReduceElems + threadIdx.x * 4;
+  const int row = idx / D, col = idx % D;
+  float4 sv = make_float4(0.f, 0.f, 0.f, 0.f), sk = sv;
+  for (int j = 0; j < tl.x; ++j) {
+    const float4 v = *reinterpret_cast<const float4*>(base + (size_t)j * 2 * tile_elems + idx);
+    const float4 k = *reinterpret_cast<const float4*>(base + (size_t)j * 2 * tile_elems + tile_elems + idx);
+    sv.x += v.x; sv.y += v.y; sv.z += v.z; sv.w += v.w;
+    sk.x += k.x; sk.y += k.y; sk.z += k.z; sk.w += k.w;
+  }
+  const long key = (long)t * kTile + row;
+  if (key >= a.Skv) return;
+  __nv_bfloat16* dvr = a.dv + b * a.dv_sb + key * a.dv_ss + (int64_t)hk * a.dv_sh + col;
+  __nv_bfloat16* dkr = a.dk + b * a.dk_sb + key * a.dk_ss + (int64_t)hk * a.dk_sh + col;
+  *reinterpret_cast<uint2*>(dvr) = make_uint2(pack_bf16x2(sv.x, sv.y), pack_bf16x2(sv.z, sv.w));
+  *reinterpret_cast<uint2*>(dkr) = make_uint2(pack_bf16x2(sk.x * a.scale, sk.y * a.scale),
+                                              pack_bf16x2(sk.z * a.scale, sk.w * a.scale));
+}
+
 // ---------------------------------------------------------------- dQ
-// TMEM columns: S [0, 128), dP [128, 256), dQ [256, 256 + D). dS (bf16 pairs)
-// replaces the first 64 columns of S. MMA order per step:
+// TMEM columns: S [0, 128), dP [128, 256), dQ [256, 256 + D). dS (bf16
+// pairs) is packed into S's columns. MMA order per step:
 // S, dP | (compute) | dQ, S(next), dP(next).
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -545,9 +708,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bar.ring_empty[i], 1);
     }
     mbar_init(&bar.mm1_ready, 1);
-    mbar_init(&bar.comp_ready, kTile);
+    mbar_init(&bar.comp_ready, kBCompute);
     mbar_init(&bar.acc_done, 1);
-    mbar_init(&bar.acc_free, kTile);
+    mbar_init(&bar.acc_free, kBCompute);
     mbar_init(&bar.final_mma, 1);
     fence_barrier_init();
   }
@@ -662,10 +825,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         if (elect_one_sync()) {
           const uint32_t kmn = ring_mn + (uint32_t)slot * 2 * kTileUnits;
-          // dQ += dS K: dS from TMEM columns [0, 64), K rows 16kk..
+          // dQ += dS K: dS packed in S's columns, K rows 16kk..
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + 256, tmem + kk * 8, sdesc_join(kmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
+            mma_ts(tmem + 256, tmem + packed_col(kk), sdesc_join(kmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
                    (s > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bar.ring_empty[slot]);
           if (!more) {
@@ -683,10 +846,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (elect_one_sync()) mma_commit(&bar.final_mma);
     __syncwarp();
     mbar_wait_timeout(&bar.final_mma, 0);
-  } else if (warp < 4) {
+  } else {
     // ------------------------------------------------------------ compute
-    const int row = threadIdx.x;  // query row of the tile = TMEM lane
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int row = threadIdx.x % kTile;  // query row of the tile = TMEM lane
+    const int half = warp / 4;            // key columns [64 half, 64 half + 64)
+    const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const float NEG_INF = -__int_as_float(0x7f800000);
     int ucnt = 0, gstep = 0;
     bool ok = true;
@@ -696,11 +860,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const QUnit w = q_unit(a, u);
       const int qi = w.qt * kTile + row;
       const bool valid = qi < a.Sq;
+      const int c_lo = half * (D / 2);
       if (w.n == 0) {
         // these queries see no key: their gradient is exactly zero
         if (valid) {
-          __nv_bfloat16* dqr = a.dq + w.b * a.dq_sb + (int64_t)qi * a.dq_ss + (int64_t)w.h * a.dq_sh;
-          for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(dqr + c) = make_uint4(0, 0, 0, 0);
+          __nv_bfloat16* dqr = a.dq + w.b * a.dq_sb + (int64_t)qi * a.dq_ss + (int64_t)w.h * a.dq_sh + c_lo;
+          for (int c = 0; c < D / 2; c += 8) *reinterpret_cast<uint4*>(dqr + c) = make_uint4(0, 0, 0, 0);
         }
         continue;
       }
@@ -723,7 +888,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         const bool full = pair_full(a, w.qt, t);
 #pragma unroll 1
-        for (int c = 0; c < kTile / 32; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * half + cc;
           float x[32], dp[32];
           tmem_ld32f(lane_base + 32 * c, x);
           tmem_ld32f(lane_base + 128 + 32 * c, dp);
@@ -743,8 +909,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             pk[e / 2] = pack_bf16x2(de[0], de[1]);
           }
-          // dS chunk c -> columns [16c, 16c + 16) (S columns already read)
-          tmem_st16(lane_base + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(pk));
+          // dS of chunk c -> the first 16 of its own 32 source columns
+          tmem_st16(lane_base + 32 * c, *reinterpret_cast<uint32_t(*)[16]>(pk));
         }
         tmem_st_wait();
         tc_fence_before();
@@ -755,11 +921,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       {
         // tcgen05.ld is warp-collective: every lane loads, only real query rows are stored
-        __nv_bfloat16* dqr = a.dq + w.b * a.dq_sb + (int64_t)(valid ? qi : 0) * a.dq_ss + (int64_t)w.h * a.dq_sh;
+        __nv_bfloat16* dqr =
+            a.dq + w.b * a.dq_sb + (int64_t)(valid ? qi : 0) * a.dq_ss + (int64_t)w.h * a.dq_sh + c_lo;
 #pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
+        for (int c = 0; c < D / 2; c += 32) {
           float q0[32];
-          tmem_ld32f(lane_base + 256 + c, q0);
+          tmem_ld32f(lane_base + 256 + c_lo + c, q0);
           tmem_ld_wait();
           reg_fence_f<32>(q0);
 #pragma unroll

@@ -242,16 +242,20 @@ attn_status attn_decode_noalloc(const attn_decode_params *p, void *stream);
  * P = exp(scale * Q K^T - LSE) over the allowed pairs:
  *   dV = P^T dO,  dS = P o (dO V^T - rowsum(dO o O)),  dQ = scale dS K,  dK = scale dS^T Q,
  * with dK and dV summed over the query heads of each KV head (GQA/MQA).
- * Three kernels: a row reduction for rowsum(dO o O) into the workspace, then
- * one tcgen05 kernel over key tiles (dK, dV) and one over query tiles (dQ).
- * Every output element is accumulated by one CTA in a fixed order with no
- * atomics, so results are bit-identical from run to run whatever
- * `deterministic` says (the flag is accepted for interface compatibility).
+ * Kernels: a row reduction for rowsum(dO o O) into the workspace (whose
+ * last block also writes the dK/dV work plan there), one tcgen05 kernel over
+ * pieces of key tiles (dK, dV; a key tile with more steps than a cap set
+ * from the work per SM is cut into pieces whose fp32 partials a reduction
+ * kernel sums in piece order) and one over query tiles (dQ). Every output
+ * element is accumulated in a fixed order with no atomics, so results are
+ * bit-identical from run to run on a device whatever `deterministic` says
+ * (the flag is accepted for interface compatibility).
  * Supported: masks NONE / CAUSAL / WINDOW, no score mod, D in {64, 128};
  * anything else returns ATTN_ERR_UNSUPPORTED. Layout rules as for attn_fwd;
- * `workspace` is caller-owned device memory of at least
- * attn_bwd_workspace_bytes(B, Hq, Sq). Sq == 0 or B == 0 launches nothing;
- * Skv == 0 gives dQ = 0 (dK, dV are empty). */
+ * `workspace` is caller-owned device memory, 16-byte aligned, of at least
+ * attn_bwd_workspace_bytes(p) bytes for the same parameters on the same
+ * device (the plan depends on the device's SM count). Sq == 0 or B == 0
+ * launches nothing; Skv == 0 gives dQ = 0 (dK, dV are empty). */
 typedef struct {
   const void *q, *k, *v, *o, *dout;  /* bf16 [B][S][H][D] via the strides below */
   const float *lse;                  /* fp32 [B][Hq][Sq] contiguous, natural log, from attn_fwd */
@@ -265,7 +269,10 @@ typedef struct {
   int *status;                       /* optional device int, ATTN_DEV_* bits */
 } attn_bwd_params;
 
-size_t attn_bwd_workspace_bytes(int B, int Hq, int Sq);
+/* Workspace bytes attn_bwd needs for these parameters on the current
+ * device: the delta rows, the dK/dV plan and the partials of split key
+ * tiles. 0 when the parameters are invalid or unsupported. */
+size_t attn_bwd_workspace_bytes(const attn_bwd_params *p);
 attn_status attn_bwd(const attn_bwd_params *p, void *workspace, size_t workspace_bytes, void *stream);
 
 /* Failure-detection self-test (no counterpart on the pages). Launches one

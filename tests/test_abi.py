@@ -82,6 +82,34 @@ def test_decode_workspace_bytes(lib):
     assert lib.attn_decode_num_splits(1, 8, 1, 100, 7) == 1  # never more splits than key tiles
 
 
+def _bwd_params(B, Hq, Hkv, S, D, mask=_lib.MASK_CAUSAL):
+    p = _lib.BwdParams()
+    p.B, p.Hq, p.Hkv, p.Sq, p.Skv, p.D = B, Hq, Hkv, S, S, D
+    p.mask.kind = mask
+    p.mask.window_left = p.mask.window_right = -1
+    return p
+
+
+def test_bwd_workspace_plan_sizes(lib):
+    # Without a GPU the library plans for 148 SMs. Causal B1 Hq32 Hkv8 S2048
+    # D128: key tile t meets 16 - t query tiles x 4 heads = 4 (16 - t) steps,
+    # 8 groups x 4 x 136 = 4352 steps, cap = ceil(4352 / (2 x 148)) = 15.
+    # Pieces per tile ceil(4 (16 - t) / 15): 5, 4 x4, 3 x4, 2 x4, 1 x3 = 44,
+    # of which 41 belong to split tiles (fp32 partial slots).
+    delta = 32 * 2048 * 4
+    pieces = 44 * 16 + 64            # 704 rounded up to 256
+    tiles = 256                      # 16 x 8 rounded up to 256
+    part = 8 * 41 * 2 * 128 * 128 * 4
+    n = lib.attn_bwd_workspace_bytes(ctypes.byref(_bwd_params(1, 32, 8, 2048, 128)))
+    assert n == delta + pieces + tiles + part
+    # no mask, one key tile per group: 1 piece each, nothing split
+    n = lib.attn_bwd_workspace_bytes(ctypes.byref(_bwd_params(2, 4, 4, 128, 64, _lib.MASK_NONE)))
+    assert n == 2 * 4 * 128 * 4 + 256 + 256
+    # unsupported: document mask, D = 96
+    assert lib.attn_bwd_workspace_bytes(ctypes.byref(_bwd_params(1, 4, 4, 128, 64, _lib.MASK_DOCUMENT))) == 0
+    assert lib.attn_bwd_workspace_bytes(ctypes.byref(_bwd_params(1, 4, 4, 128, 96))) == 0
+
+
 def _fwd_params(**kw):
     p = _lib.FwdParams()
     p.q = p.k = p.v = p.o = 1 << 20

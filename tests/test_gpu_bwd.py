@@ -92,6 +92,14 @@ def test_bwd_explicit_scale():
     bwd_case(1, 256, 2, 2, 128, seed=230, causal=True, scale=0.3)
 
 
+def test_bwd_split_key_tiles():
+    # small causal problems get a piece cap of 4 steps, so most key tiles are
+    # cut into several pieces whose fp32 partials the reduction sums
+    bwd_case(1, 1024, 8, 2, 128, seed=250, causal=True)
+    bwd_case(2, 700, 4, 1, 64, seed=251, causal=True)
+    bwd_case(1, 900, 6, 2, 128, Skv=1300, seed=252, window=(300, 40), q_offset=200)
+
+
 def test_bwd_full_size_causal_gqa():
     w = W.WORKLOADS["causal_gqa_llama8b_s2048"]
     bwd_case(w.B, w.S, w.Hq, w.Hkv, w.D, seed=w.seed, causal=True)
