@@ -322,3 +322,72 @@ def attn_bwd(q, k, v, dout, *, scale: Optional[float] = None, mask: int = MASK_N
     if lib.oracle_attn_bwd_f64(ctypes.byref(a), dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, nt) != 0:
         raise ValueError("oracle_attn_bwd_f64: bad arguments")
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------- kv-cache update
+# FlashAttention overview ("Examples", flash_attn_with_kvcache): new keys and
+# values are written into the cache in place, and rotary embeddings
+# (rotary_cos, rotary_sin, rotary_interleaved) are applied on the fly. The
+# pages give only the argument list; the readings used here:
+#  - the new tokens of sequence b take cache positions cache_seqlens[b] + i,
+#    i = 0 .. Snew - 1, and their rotary position is that same cache position,
+#    for q and for the new k alike; v is not rotated;
+#  - the rotary tables hold cos / sin of angle j at each position, shape
+#    [positions, rotary_dim / 2]; pair j of a head vector is (x[2j], x[2j+1])
+#    when interleaved, else (x[j], x[j + rotary_dim / 2]); dims past
+#    rotary_dim are left unchanged;
+#  - a paged cache maps position p of sequence b to page
+#    block_table[b][p // page_size], row p % page_size; a contiguous cache
+#    [B_cache][S][Hkv][D] maps it to batch row cache_batch_idx[b] (or b).
+
+
+def rotary(x, cos, sin, positions, interleaved: bool):
+    """Rotates the first 2 * cos.shape[1] dims of x[..., t, h, :] by the angles at
+    positions[..., t]: x float64 [B, T, H, D]; cos, sin float64 [P, R/2];
+    positions int [B, T]. Returns a new float64 array."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    half = cos.shape[1]
+    c = cos[positions][:, :, None, :]  # [B, T, 1, R/2]
+    s = sin[positions][:, :, None, :]
+    if interleaved:
+        a, b = x[..., 0:2 * half:2].copy(), x[..., 1:2 * half:2].copy()
+        x[..., 0:2 * half:2] = a * c - b * s
+        x[..., 1:2 * half:2] = a * s + b * c
+    else:
+        a, b = x[..., :half].copy(), x[..., half:2 * half].copy()
+        x[..., :half] = a * c - b * s
+        x[..., half:2 * half] = a * s + b * c
+    return x
+
+
+def cache_rows(B: int, Snew: int, cache_seqlens, block_table=None, page_size: int = 0, cache_batch_idx=None):
+    """(page or batch row, slot) of every new token: arrays [B, Snew] each."""
+    pos = np.asarray(cache_seqlens, dtype=np.int64)[:, None] + np.arange(Snew, dtype=np.int64)[None, :]
+    if block_table is not None:
+        bt = np.asarray(block_table, dtype=np.int64)
+        return bt[np.arange(B)[:, None], pos // page_size], pos % page_size
+    idx = np.arange(B) if cache_batch_idx is None else np.asarray(cache_batch_idx, dtype=np.int64)
+    return np.broadcast_to(idx[:, None], pos.shape).copy(), pos
+
+
+def kvcache_append(k_cache, v_cache, k_new, v_new, cache_seqlens, *, block_table=None, page_size: int = 0,
+                   cache_batch_idx=None, rotary_cos=None, rotary_sin=None, interleaved: bool = True,
+                   round_bf16=None):
+    """Returns updated copies of k_cache / v_cache (float64, same shapes) with the
+    new tokens written at their cache positions, k rotated when tables are
+    given. round_bf16, when given, rounds the rotated k to the cache's storage
+    type before it is stored (the update writes bf16)."""
+    kc, vc = np.array(k_cache, dtype=np.float64, copy=True), np.array(v_cache, dtype=np.float64, copy=True)
+    B, Snew = k_new.shape[0], k_new.shape[1]
+    pos = np.asarray(cache_seqlens, dtype=np.int64)[:, None] + np.arange(Snew, dtype=np.int64)[None, :]
+    k = np.asarray(k_new, dtype=np.float64)
+    if rotary_cos is not None:
+        k = rotary(k, rotary_cos, rotary_sin, pos, interleaved)
+    if round_bf16 is not None:
+        k = round_bf16(k)
+    row, slot = cache_rows(B, Snew, cache_seqlens, block_table, page_size, cache_batch_idx)
+    for b in range(B):
+        for i in range(Snew):
+            kc[row[b, i], slot[b, i]] = k[b, i]
+            vc[row[b, i], slot[b, i]] = v_new[b, i]
+    return kc, vc
