@@ -25,7 +25,7 @@ from ._lib import (ATTN_DEV_BAD_LEN, ATTN_DEV_BAD_MASK, ATTN_DEV_BAD_PAGE, ATTN_
                    MASK_DOCUMENT, MASK_NONE, MASK_WINDOW,
                    MOD_ALIBI, MOD_NONE, MOD_SOFTCAP, AttnError)
 
-__all__ = ["attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_decode", "attn_decode_noalloc", "attn_build_block_mask", "attn_lse_combine",
+__all__ = ["attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_kvcache_update", "attn_with_kvcache", "attn_decode", "attn_decode_noalloc", "attn_build_block_mask", "attn_lse_combine",
            "BlockMask", "AttnError",
            "load_library", "ATTN_DEV_TIMEOUT", "ATTN_DEV_BAD_PAGE", "ATTN_DEV_BAD_LEN",
            "ATTN_DEV_BAD_MASK"]
@@ -294,38 +294,54 @@ def attn_bwd(q, k, v, out, lse, dout, *, scale: Optional[float] = None, causal: 
 
 
 def _decode_params(q, k_cache, v_cache, block_table, cache_seqlens, max_seqlen, scale, softcap, alibi_slopes,
-                   num_splits, out, lse, status):
+                   num_splits, out, lse, status, causal=False, cache_batch_idx=None):
     """Checks the decode inputs and fills the C parameter block (shared by
-    attn_decode and attn_decode_noalloc)."""
+    attn_decode and attn_decode_noalloc). q is [B, Hq, D] or [B, q_len, Hq, D];
+    block_table None selects a contiguous cache [rows, positions, Hkv, D]."""
     torch = _torch()
+    q_len = 1
     if q.dim() == 4:
-        q = q[:, 0]
-    _check_bf16("q", q, 3)
+        q_len = q.shape[1]
+        if q_len == 1:
+            q = q[:, 0]
+    _check_bf16("q", q, 4 if q_len > 1 else 3)
     _check_bf16("k_cache", k_cache, 4)
     _check_bf16("v_cache", v_cache, 4)
     if k_cache.shape != v_cache.shape or k_cache.stride() != v_cache.stride():
         raise ValueError("k_cache and v_cache must share shape and strides")
-    for name, t in (("block_table", block_table), ("cache_seqlens", cache_seqlens)):
-        if t.dtype != torch.int32 or not t.is_cuda:
-            raise ValueError("%s must be an int32 CUDA tensor" % name)
-    if block_table.dim() != 2 or block_table.stride(1) != 1 or not cache_seqlens.is_contiguous():
-        raise ValueError("block_table rows and cache_seqlens must be contiguous")
-    B, Hq, D = q.shape
+    tables = [("cache_seqlens", cache_seqlens)]
+    if block_table is not None:
+        tables.append(("block_table", block_table))
+    if cache_batch_idx is not None:
+        tables.append(("cache_batch_idx", cache_batch_idx))
+    for name, t in tables:
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous int32 CUDA tensor" % name)
+    B, Hq, D = q.shape[0], q.shape[-2], q.shape[-1]
     P, page, Hkv, Dk = k_cache.shape
-    if Dk != D or block_table.shape[0] != B or cache_seqlens.numel() != B:
+    if Dk != D or cache_seqlens.numel() != B or (block_table is not None and block_table.shape[0] != B):
         raise ValueError("q, caches, block_table and cache_seqlens disagree on B or D")
-    if out is not None and (tuple(out.shape) != (B, Hq, D) or out.dtype != torch.bfloat16):
-        raise ValueError("out must be bf16 [B, Hq, D]")
-    if lse is not None and (tuple(lse.shape) != (B, Hq) or lse.dtype != torch.float32 or not lse.is_contiguous()):
-        raise ValueError("lse must be contiguous fp32 [B, Hq]")
+    if cache_batch_idx is not None and (block_table is not None or cache_batch_idx.numel() != B):
+        raise ValueError("cache_batch_idx needs a contiguous cache (no block_table) and B entries")
+    oshape = (B, Hq, D) if q_len == 1 else (B, q_len, Hq, D)
+    if out is not None and (tuple(out.shape) != oshape or out.dtype != torch.bfloat16):
+        raise ValueError("out must be bf16 %s" % (oshape,))
+    lshape = (B, Hq) if q_len == 1 else (B, q_len, Hq)
+    if lse is not None and (tuple(lse.shape) != lshape or lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise ValueError("lse must be contiguous fp32 %s" % (lshape,))
     if max_seqlen is None:
-        max_seqlen = block_table.shape[1] * page
+        max_seqlen = block_table.shape[1] * page if block_table is not None else page
     p = _lib.DecodeParams()
     p.q = q.data_ptr()
-    p.q_stride = _lib.c_i64x2(q.stride(0), q.stride(1))
+    p.q_stride = _lib.c_i64x2(q.stride(0), q.stride(-2))
+    p.q_len = q_len
+    p.q_token_stride = q.stride(1) if q_len > 1 else 0
+    p.causal = 1 if causal else 0
     p.k_cache, p.v_cache = k_cache.data_ptr(), v_cache.data_ptr()
     p.cache_stride = _lib.c_i64x3(*k_cache.stride()[:3])
-    p.block_table, p.block_table_stride = block_table.data_ptr(), block_table.stride(0)
+    if block_table is not None:
+        p.block_table, p.block_table_stride = block_table.data_ptr(), block_table.stride(0)
+    p.cache_batch_idx = _ptr(cache_batch_idx)
     p.cache_seqlens = cache_seqlens.data_ptr()
     p.B, p.Hq, p.Hkv, p.D, p.page_size, p.num_pages = B, Hq, Hkv, D, page, P
     p.max_seqlen = int(max_seqlen)
@@ -337,28 +353,39 @@ def _decode_params(q, k_cache, v_cache, block_table, cache_seqlens, max_seqlen, 
     return p, q
 
 
+def _set_out(p, out):
+    p.o = out.data_ptr()
+    p.o_stride = _lib.c_i64x2(out.stride(0), out.stride(-2))
+    p.o_token_stride = out.stride(1) if p.q_len > 1 else 0
+
+
 def attn_decode(q, k_cache, v_cache, block_table, cache_seqlens, *, max_seqlen: Optional[int] = None,
                 scale: Optional[float] = None, softcap: Optional[float] = None, alibi_slopes=None,
                 num_splits: int = 0, out=None, lse=None, workspace=None, status=None, with_lse: bool = True,
-                stream=None):
-    """Split-KV decode over a paged cache. q [B, Hq, D] (or [B, 1, Hq, D]);
-    k_cache/v_cache [num_pages, page_size, Hkv, D]; block_table int32
-    [B, max_pages]; cache_seqlens int32 [B]. Returns (O [B, Hq, D], LSE [B, Hq])."""
+                causal: bool = False, cache_batch_idx=None, stream=None):
+    """Split-KV decode over a KV cache. q [B, Hq, D], or [B, q_len, Hq, D] for
+    several new tokens per sequence (they are the last q_len positions;
+    `causal` masks each token's later keys); k_cache/v_cache
+    [num_pages, page_size, Hkv, D] with block_table int32 [B, max_pages], or
+    a contiguous cache [rows, positions, Hkv, D] with block_table None and
+    optional cache_batch_idx int32 [B]; cache_seqlens int32 [B] counts every
+    key, new tokens included. Returns O [B, Hq, D] for one token, else
+    [B, q_len, Hq, D], and LSE [B, Hq] or [B, q_len, Hq]."""
     torch = _torch()
     B, Hq, D = (q.shape[0], q.shape[-2], q.shape[-1])
-    if out is None:
-        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    q_len = q.shape[1] if q.dim() == 4 else 1
+    if out is None:  # one token: [B, Hq, D] whether q came as [B, Hq, D] or [B, 1, Hq, D]
+        out = torch.empty((B, Hq, D) if q_len == 1 else (B, q_len, Hq, D), dtype=torch.bfloat16, device=q.device)
     if lse is None and with_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, Hq) if q_len == 1 else (B, q_len, Hq), dtype=torch.float32, device=q.device)
     p, q = _decode_params(q, k_cache, v_cache, block_table, cache_seqlens, max_seqlen, scale, softcap,
-                          alibi_slopes, num_splits, out, lse, status)
+                          alibi_slopes, num_splits, out, lse, status, causal, cache_batch_idx)
     lib = _lib.load()
     splits = lib.attn_decode_num_splits(p.B, p.Hq, p.Hkv, p.max_seqlen, p.num_splits)
-    need = lib.attn_decode_workspace_bytes(p.B, p.Hq, p.D, splits)
+    need = lib.attn_decode_workspace_bytes(p.B, p.Hq * p.q_len, p.D, splits)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    p.o = out.data_ptr()
-    p.o_stride = _lib.c_i64x2(out.stride(0), out.stride(1))
+    _set_out(p, out)
     h = _stream_handle(q.device) if stream is None else stream
     _lib.check(lib.attn_decode(ctypes.byref(p), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                h), "attn_decode")
@@ -367,19 +394,102 @@ def attn_decode(q, k_cache, v_cache, block_table, cache_seqlens, *, max_seqlen: 
 
 def attn_decode_noalloc(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, *, max_seqlen: int,
                         scale: Optional[float] = None, softcap: Optional[float] = None, alibi_slopes=None,
-                        num_splits: int = 0, status=None, stream=None):
+                        num_splits: int = 0, status=None, causal: bool = False, cache_batch_idx=None, stream=None):
     """attn_decode whose split partials live in a fixed 32 MiB array inside the
     library, for callers that may not allocate device memory (out and lse are
     the caller's). Calls that would need more scratch raise AttnError
     (workspace too small). The first call on a device should precede any
     stream capture; calls that overlap on the GPU share the array and race."""
     p, q = _decode_params(q, k_cache, v_cache, block_table, cache_seqlens, max_seqlen, scale, softcap,
-                          alibi_slopes, num_splits, out, lse, status)
-    p.o = out.data_ptr()
-    p.o_stride = _lib.c_i64x2(out.stride(0), out.stride(1))
+                          alibi_slopes, num_splits, out, lse, status, causal, cache_batch_idx)
+    _set_out(p, out)
     h = _stream_handle(q.device) if stream is None else stream
     _lib.check(_lib.load().attn_decode_noalloc(ctypes.byref(p), h), "attn_decode_noalloc")
     return out, lse
+
+
+def attn_kvcache_update(k_cache, v_cache, cache_seqlens, *, q=None, q_out=None, k=None, v=None, block_table=None,
+                        cache_batch_idx=None, rotary_cos=None, rotary_sin=None, rotary_interleaved: bool = True,
+                        seqlens_out=None, status=None, stream=None):
+    """In-place cache update of flash_attn_with_kvcache: k/v [B, Snew, Hkv, D]
+    (k rotated) are written at positions cache_seqlens[b] + i of the paged
+    (block_table) or contiguous (cache_batch_idx) cache, q [B, Snew, Hq, D]
+    rotated at the same positions into q_out (allocated when None, may be q).
+    rotary_cos / rotary_sin: fp32 [positions, rotary_dim / 2]. Returns q_out."""
+    torch = _torch()
+    _check_bf16("k_cache", k_cache, 4)
+    _check_bf16("v_cache", v_cache, 4)
+    if k_cache.shape != v_cache.shape or k_cache.stride() != v_cache.stride():
+        raise ValueError("k_cache and v_cache must share shape and strides")
+    P, page, Hkv, D = k_cache.shape
+    ref = q if q is not None else k
+    if ref is None:
+        raise ValueError("nothing to update: give q and/or k, v")
+    B, Snew = ref.shape[0], ref.shape[1]
+    p = _lib.KvUpdateParams()
+    if q is not None:
+        _check_bf16("q", q, 4)
+        if q_out is None:
+            q_out = torch.empty_like(q)
+        p.q, p.q_out = q.data_ptr(), q_out.data_ptr()
+        p.q_stride, p.q_out_stride = _lib.c_i64x3(*q.stride()[:3]), _lib.c_i64x3(*q_out.stride()[:3])
+        p.Hq = q.shape[2]
+    else:
+        p.q_stride = p.q_out_stride = _lib.c_i64x3(8, 8, 8)
+    if (k is None) != (v is None):
+        raise ValueError("give k and v together")
+    if k is not None:
+        _check_bf16("k", k, 4)
+        _check_bf16("v", v, 4)
+        p.k_new, p.v_new = k.data_ptr(), v.data_ptr()
+        p.k_new_stride, p.v_new_stride = _lib.c_i64x3(*k.stride()[:3]), _lib.c_i64x3(*v.stride()[:3])
+    else:
+        p.k_new_stride = p.v_new_stride = _lib.c_i64x3(8, 8, 8)
+    p.k_cache, p.v_cache = k_cache.data_ptr(), v_cache.data_ptr()
+    p.cache_stride = _lib.c_i64x3(*k_cache.stride()[:3])
+    if block_table is not None:
+        p.block_table, p.block_table_stride = block_table.data_ptr(), block_table.stride(0)
+    p.cache_batch_idx = _ptr(cache_batch_idx)
+    p.cache_seqlens = cache_seqlens.data_ptr()
+    p.seqlens_out = _ptr(seqlens_out)
+    p.B, p.Snew, p.Hkv, p.D, p.page_size, p.num_pages = B, Snew, Hkv, D, page, P
+    if rotary_cos is not None:
+        if rotary_cos.dtype != torch.float32 or rotary_sin is None or rotary_sin.dtype != torch.float32:
+            raise ValueError("rotary_cos / rotary_sin must be fp32 [positions, rotary_dim / 2]")
+        if not (rotary_cos.is_contiguous() and rotary_sin.is_contiguous()) or rotary_cos.shape != rotary_sin.shape:
+            raise ValueError("rotary tables must be contiguous and of one shape")
+        p.rotary_cos, p.rotary_sin = rotary_cos.data_ptr(), rotary_sin.data_ptr()
+        p.rotary_positions, p.rotary_dim = rotary_cos.shape[0], 2 * rotary_cos.shape[1]
+    p.rotary_interleaved = 1 if rotary_interleaved else 0
+    p.status = _ptr(status)
+    h = _stream_handle(k_cache.device) if stream is None else stream
+    _lib.check(_lib.load().attn_kvcache_update(ctypes.byref(p), h), "attn_kvcache_update")
+    return q_out
+
+
+def attn_with_kvcache(q, k_cache, v_cache, cache_seqlens, *, k=None, v=None, rotary_cos=None, rotary_sin=None,
+                      cache_batch_idx=None, block_table=None, softmax_scale: Optional[float] = None,
+                      causal: bool = False, rotary_interleaved: bool = True, alibi_slopes=None,
+                      softcap: Optional[float] = None, num_splits: int = 0, max_seqlen: Optional[int] = None,
+                      status=None, stream=None):
+    """flash_attn_with_kvcache (FlashAttention overview, "Examples"): optional
+    in-place append of k/v with rotary embedding (attn_kvcache_update), then
+    attention of q [B, Sq, Hq, D] over each sequence's cache, the Sq new
+    tokens at its last positions. Returns (O [B, Sq, Hq, D], LSE [B, Sq, Hq])."""
+    torch = _torch()
+    seqlens = cache_seqlens
+    if k is not None or rotary_cos is not None:
+        seqlens = torch.empty_like(cache_seqlens) if k is not None else cache_seqlens
+        q = attn_kvcache_update(k_cache, v_cache, cache_seqlens, q=q, k=k, v=v, block_table=block_table,
+                                cache_batch_idx=cache_batch_idx, rotary_cos=rotary_cos, rotary_sin=rotary_sin,
+                                rotary_interleaved=rotary_interleaved,
+                                seqlens_out=seqlens if k is not None else None, status=status, stream=stream)
+    if max_seqlen is None:
+        page = k_cache.shape[1]
+        max_seqlen = block_table.shape[1] * page if block_table is not None else page
+    return attn_decode(q, k_cache, v_cache, block_table, seqlens, max_seqlen=max_seqlen, scale=softmax_scale,
+                       softcap=softcap, alibi_slopes=alibi_slopes, num_splits=num_splits, causal=causal,
+                       cache_batch_idx=cache_batch_idx, status=status, stream=stream)
 
 
 def attn_lse_combine(o_parts, lse_parts, *, out=None, lse=None, stream=None):

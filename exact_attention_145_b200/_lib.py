@@ -28,7 +28,7 @@ MOD_NONE, MOD_SOFTCAP, MOD_ALIBI = range(3)
 EXPORTS = ("attn_block_mask_bytes", "attn_block_mask_layout", "attn_build_block_mask", "attn_fwd",
            "attn_decode_num_splits", "attn_decode_workspace_bytes", "attn_decode", "attn_lse_combine",
            "attn_status_str", "attn_decode_noalloc", "attn_selftest_wait_timeout", "attn_bwd_workspace_bytes",
-           "attn_bwd")
+           "attn_bwd", "attn_kvcache_update")
 ATTN_DECODE_NOALLOC_MAX_BYTES = 32 * 1024 * 1024
 
 c_i64x3 = ctypes.c_int64 * 3
@@ -82,6 +82,22 @@ class DecodeParams(ctypes.Structure):
                 ("alibi_slopes", ctypes.c_void_p), ("alibi_batch_stride", ctypes.c_int),
                 ("num_splits", ctypes.c_int),
                 ("o", ctypes.c_void_p), ("o_stride", c_i64x2), ("lse", ctypes.c_void_p),
+                ("status", ctypes.c_void_p),
+                ("q_len", ctypes.c_int), ("q_token_stride", ctypes.c_int64), ("o_token_stride", ctypes.c_int64),
+                ("causal", ctypes.c_int), ("cache_batch_idx", ctypes.c_void_p)]
+
+
+class KvUpdateParams(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("q_stride", c_i64x3), ("q_out", ctypes.c_void_p), ("q_out_stride", c_i64x3),
+                ("k_new", ctypes.c_void_p), ("v_new", ctypes.c_void_p), ("k_new_stride", c_i64x3),
+                ("v_new_stride", c_i64x3), ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("cache_stride", c_i64x3), ("block_table", ctypes.c_void_p), ("block_table_stride", ctypes.c_int),
+                ("cache_batch_idx", ctypes.c_void_p), ("cache_seqlens", ctypes.c_void_p),
+                ("seqlens_out", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("Snew", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("D", ctypes.c_int), ("page_size", ctypes.c_int), ("num_pages", ctypes.c_int),
+                ("rotary_cos", ctypes.c_void_p), ("rotary_sin", ctypes.c_void_p), ("rotary_dim", ctypes.c_int),
+                ("rotary_positions", ctypes.c_int), ("rotary_interleaved", ctypes.c_int),
                 ("status", ctypes.c_void_p)]
 
 
@@ -122,6 +138,8 @@ def load() -> ctypes.CDLL:
         lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.attn_bwd.argtypes = [ctypes.POINTER(BwdParams), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
         lib.attn_bwd.restype = ctypes.c_int
+        lib.attn_kvcache_update.argtypes = [ctypes.POINTER(KvUpdateParams), ctypes.c_void_p]
+        lib.attn_kvcache_update.restype = ctypes.c_int
         lib.attn_lse_combine.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
         lib.attn_lse_combine.restype = ctypes.c_int

@@ -14,6 +14,7 @@
 #include "aux_kernels.cuh"
 #include "bwd_kernel.cuh"
 #include "fwd_kernel.cuh"
+#include "kvcache_kernel.cuh"
 
 using namespace attn_kernels;
 
@@ -54,8 +55,10 @@ void set_trace(FwdArgs& a) {
 
 // A bf16 tensor map over (dims[0] contiguous, dims[1..r-1] with element
 // strides), box = {64, box_rows, 1, ...}, 128-byte swizzle.
+// Tiled bf16 map with a 64-column inner box (SW128); box_rows rows along
+// dimension box_rows_dim and, when box2_dim > 0, box2_rows along box2_dim.
 attn_status make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const int64_t* strides_el,
-                     uint32_t box_rows, int box_rows_dim) {
+                     uint32_t box_rows, int box_rows_dim, uint32_t box2_rows = 1, int box2_dim = 0) {
   auto enc = encoder();
   if (!enc) return ATTN_ERR_CUDA;
   cuuint64_t gdim[5];
@@ -70,6 +73,7 @@ attn_status make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
   }
   box[0] = 64;
   box[box_rows_dim] = box_rows;
+  if (box2_dim > 0) box[box2_dim] = box2_rows;
   for (int i = 1; i < rank; ++i) {
     const int64_t b = strides_el[i - 1] * 2;
     if (b <= 0 || (b % 16) != 0 || b >= (1ll << 40)) return ATTN_ERR_UNSUPPORTED;
@@ -368,6 +372,80 @@ attn_status attn_bwd(const attn_bwd_params* p, void* workspace, size_t workspace
   return p->D == 128 ? launch_bwd<128>(mq, mk, mv, mdo, a, st) : launch_bwd<64>(mq, mk, mv, mdo, a, st);
 }
 
+attn_status attn_kvcache_update(const attn_kvcache_update_params* p, void* stream) {
+  using namespace attn_kv_kernels;
+  if (!p) return ATTN_ERR_INVALID_ARG;
+  if (p->B < 0 || p->Snew < 0 || p->Hq < 0 || p->Hkv < 0 || p->page_size <= 0 || p->num_pages <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (p->D != 64 && p->D != 128) return ATTN_ERR_UNSUPPORTED;
+  const bool has_q = p->q != nullptr, has_kv = p->k_new != nullptr;
+  if (has_kv != (p->v_new != nullptr) || (has_q && !p->q_out) || (has_kv && (!p->k_cache || !p->v_cache)))
+    return ATTN_ERR_INVALID_ARG;
+  if (!p->cache_seqlens) return ATTN_ERR_INVALID_ARG;
+  if (p->block_table && p->block_table_stride <= 0) return ATTN_ERR_INVALID_ARG;
+  if (p->rotary_cos || p->rotary_sin) {
+    if (!p->rotary_cos || !p->rotary_sin || p->rotary_positions <= 0) return ATTN_ERR_INVALID_ARG;
+    if (p->rotary_dim <= 0 || p->rotary_dim % 16 != 0 || p->rotary_dim > p->D) return ATTN_ERR_UNSUPPORTED;
+  }
+  const void* ptrs[] = {p->q, p->q_out, p->k_new, p->v_new, p->k_cache, p->v_cache};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return ATTN_ERR_UNSUPPORTED;
+  const int64_t* strides[] = {p->q_stride, p->q_out_stride, p->k_new_stride, p->v_new_stride, p->cache_stride};
+  for (const int64_t* st : strides)
+    if (!strides_ok(st, 3)) return ATTN_ERR_UNSUPPORTED;
+  if (p->B == 0) return ATTN_OK;
+  KvUpdateArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(p->q);
+  a.q_sb = p->q_stride[0];
+  a.q_ss = p->q_stride[1];
+  a.q_sh = p->q_stride[2];
+  a.q_out = static_cast<__nv_bfloat16*>(p->q_out);
+  a.qo_sb = p->q_out_stride[0];
+  a.qo_ss = p->q_out_stride[1];
+  a.qo_sh = p->q_out_stride[2];
+  a.k_new = static_cast<const __nv_bfloat16*>(p->k_new);
+  a.v_new = static_cast<const __nv_bfloat16*>(p->v_new);
+  a.kn_sb = p->k_new_stride[0];
+  a.kn_ss = p->k_new_stride[1];
+  a.kn_sh = p->k_new_stride[2];
+  a.vn_sb = p->v_new_stride[0];
+  a.vn_ss = p->v_new_stride[1];
+  a.vn_sh = p->v_new_stride[2];
+  a.k_cache = static_cast<__nv_bfloat16*>(p->k_cache);
+  a.v_cache = static_cast<__nv_bfloat16*>(p->v_cache);
+  a.c_sp = p->cache_stride[0];
+  a.c_ss = p->cache_stride[1];
+  a.c_sh = p->cache_stride[2];
+  a.block_table = p->block_table;
+  a.bt_stride = p->block_table_stride;
+  a.cache_batch_idx = p->block_table ? nullptr : p->cache_batch_idx;
+  a.seqlens = p->cache_seqlens;
+  a.seqlens_out = p->seqlens_out;
+  a.B = p->B;
+  a.Snew = p->Snew;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.D = p->D;
+  a.page_size = p->page_size;
+  a.num_pages = p->num_pages;
+  a.cos = p->rotary_cos;
+  a.sin = p->rotary_sin;
+  a.rot_dim = p->rotary_cos ? p->rotary_dim : 0;
+  a.rot_positions = p->rotary_positions;
+  a.interleaved = p->rotary_interleaved ? 1 : 0;
+  a.status = p->status;
+  const int64_t q_rows = has_q ? (int64_t)p->B * p->Snew * p->Hq : 0;
+  const int64_t kv_rows = has_kv ? (int64_t)p->B * p->Snew * p->Hkv : 0;
+  if (q_rows > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+  a.q_rows = (int)q_rows;
+  int64_t threads = (q_rows + kv_rows) * (p->D / 8);
+  if (threads < p->B) threads = p->B;  // seqlens_out
+  const int64_t blocks = (threads + 255) / 256;
+  if (blocks > 0x7fffffffL) return ATTN_ERR_UNSUPPORTED;
+  kvcache_update_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 const char* attn_status_str(attn_status s) {
   switch (s) {
     case ATTN_OK:
@@ -658,22 +736,26 @@ attn_status attn_decode(const attn_decode_params* p, void* workspace, size_t wor
   if (p->B < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->page_size <= 0 || p->num_pages <= 0) return ATTN_ERR_INVALID_ARG;
   if (p->Hq % p->Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (p->D != 64 && p->D != 128) return ATTN_ERR_UNSUPPORTED;
-  if (p->Hq / p->Hkv > kRows) return ATTN_ERR_UNSUPPORTED;
-  if (p->page_size % 16 != 0 || (p->page_size < kKeys && kKeys % p->page_size != 0) ||
-      (p->page_size > kKeys && p->page_size % kKeys != 0))
+  const int q_len = p->q_len > 1 ? p->q_len : 1;
+  const bool paged = p->block_table != nullptr;
+  if (p->q_len < 0) return ATTN_ERR_INVALID_ARG;
+  if ((p->Hq / p->Hkv) * q_len > kRows) return ATTN_ERR_UNSUPPORTED;
+  if (paged && (p->page_size % 16 != 0 || (p->page_size < kKeys && kKeys % p->page_size != 0) ||
+                (p->page_size > kKeys && p->page_size % kKeys != 0)))
     return ATTN_ERR_UNSUPPORTED;
   if (p->B == 0) return ATTN_OK;
-  if (!p->q || !p->k_cache || !p->v_cache || !p->block_table || !p->cache_seqlens || !p->o)
-    return ATTN_ERR_INVALID_ARG;
-  if (p->max_seqlen <= 0 || p->block_table_stride <= 0) return ATTN_ERR_INVALID_ARG;
-  if ((long)p->block_table_stride * p->page_size < p->max_seqlen) return ATTN_ERR_INVALID_ARG;
+  if (!p->q || !p->k_cache || !p->v_cache || !p->cache_seqlens || !p->o) return ATTN_ERR_INVALID_ARG;
+  if (p->max_seqlen <= 0 || (paged && p->block_table_stride <= 0)) return ATTN_ERR_INVALID_ARG;
+  if ((long)(paged ? p->block_table_stride : 1) * p->page_size < p->max_seqlen) return ATTN_ERR_INVALID_ARG;
+  if (q_len > 1 && (p->q_token_stride <= 0 || p->o_token_stride <= 0 || (p->q_token_stride % 8) != 0))
+    return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->o))
     return ATTN_ERR_UNSUPPORTED;
   if (!strides_ok(p->q_stride, 2) || !strides_ok(p->cache_stride, 3) || !strides_ok(p->o_stride, 2))
     return ATTN_ERR_UNSUPPORTED;
   if (attn_status st = check_mods(p->mod, p->softcap, p->alibi_slopes, p->alibi_batch_stride, p->Hq)) return st;
   const int splits = attn_decode_num_splits(p->B, p->Hq, p->Hkv, p->max_seqlen, p->num_splits);
-  const size_t need = attn_decode_workspace_bytes(p->B, p->Hq, p->D, splits);
+  const size_t need = attn_decode_workspace_bytes(p->B, p->Hq * q_len, p->D, splits);
   if (!workspace || !aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
   if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
 
@@ -692,16 +774,22 @@ attn_status attn_decode(const attn_decode_params* p, void* workspace, size_t wor
   a.alibi_bstride = p->alibi_batch_stride;
   a.status = p->status;
   a.block_table = p->block_table;
-  a.bt_stride = p->block_table_stride;
+  a.cache_batch_idx = paged ? nullptr : p->cache_batch_idx;
+  a.bt_stride = paged ? p->block_table_stride : 1;
   a.seqlens = p->cache_seqlens;
   a.page_size = p->page_size;
   a.num_pages = p->num_pages;
-  a.box_rows = p->page_size < kKeys ? p->page_size : kKeys;
+  a.box_rows = (paged && p->page_size < kKeys) ? p->page_size : kKeys;
+  a.q_len = q_len;
+  a.q_causal = q_len > 1 && p->causal ? 1 : 0;
+  const int g = p->Hq / p->Hkv;
+  const int tok_box = kRows / g;  // >= q_len
+  a.q_bytes = (q_len > 1 ? g * tok_box : kRows) * p->D * 2;
   const int tiles = (p->max_seqlen + kKeys - 1) / kKeys;
   a.n_splits = splits;
   a.tiles_per_split = (tiles + splits - 1) / splits;
   a.max_seqlen = p->max_seqlen;
-  const size_t rows = (size_t)p->B * p->Hq * splits;
+  const size_t rows = (size_t)p->B * q_len * p->Hq * splits;
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((rows * p->D * 4 + 255) & ~size_t(255)));
 
@@ -711,7 +799,15 @@ attn_status attn_decode(const attn_decode_params* p, void* workspace, size_t wor
   const uint64_t dc[4] = {(uint64_t)p->D, (uint64_t)p->Hkv, (uint64_t)p->page_size, (uint64_t)p->num_pages};
   const int64_t sc[3] = {p->cache_stride[2] > 0 ? p->cache_stride[2] : 8, p->cache_stride[1],
                          p->cache_stride[0]};
-  if (attn_status st = make_map(&mq, p->q, 3, dq, sq, kRows, 1)) return st;
+  if (q_len > 1) {
+    // dims (D, g, Hkv, q_len, B), box (64, g, 1, 128 / g, 1): token i's heads land at rows i*g ..
+    const uint64_t dq5[5] = {(uint64_t)p->D, (uint64_t)g, (uint64_t)p->Hkv, (uint64_t)q_len, (uint64_t)p->B};
+    const int64_t sh = p->q_stride[1] > 0 ? p->q_stride[1] : 8;
+    const int64_t sq5[4] = {sh, sh * g, p->q_token_stride, p->q_stride[0] > 0 ? p->q_stride[0] : 8};
+    if (attn_status st = make_map(&mq, p->q, 5, dq5, sq5, (uint32_t)g, 1, (uint32_t)tok_box, 3)) return st;
+  } else if (attn_status st = make_map(&mq, p->q, 3, dq, sq, kRows, 1)) {
+    return st;
+  }
   if (attn_status st = make_map(&mk, p->k_cache, 4, dc, sc, (uint32_t)a.box_rows, 2)) return st;
   if (attn_status st = make_map(&mv, p->v_cache, 4, dc, sc, (uint32_t)a.box_rows, 2)) return st;
 
@@ -728,12 +824,14 @@ attn_status attn_decode(const attn_decode_params* p, void* workspace, size_t wor
   CombineArgs c;
   c.o_parts = a.part_o;
   c.lse_parts = a.part_lse;
-  c.rows = p->B * p->Hq;
+  c.rows = p->B * q_len * p->Hq;
   c.n = splits;
   c.D = p->D;
-  c.rows_per_b = p->Hq;
+  c.rows_per_b = q_len * p->Hq;
+  c.heads = p->Hq;
   c.o = static_cast<__nv_bfloat16*>(p->o);
   c.o_sb = p->o_stride[0];
+  c.o_st = q_len > 1 ? p->o_token_stride : 0;
   c.o_sh = p->o_stride[1];
   c.lse = p->lse;
   return launch_combine(c, p->D, s);
@@ -754,8 +852,10 @@ attn_status attn_lse_combine(const float* o_parts, const float* lse_parts, int r
   c.n = n_splits;
   c.D = D;
   c.rows_per_b = rows;
+  c.heads = rows > 0 ? rows : 1;
   c.o = static_cast<__nv_bfloat16*>(o);
   c.o_sb = 0;
+  c.o_st = 0;
   c.o_sh = o_row_stride;
   c.lse = lse;
   return launch_combine(c, D, static_cast<cudaStream_t>(stream));

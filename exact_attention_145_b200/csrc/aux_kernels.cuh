@@ -272,9 +272,10 @@ struct CombineArgs {
   const float* o_parts;    // [rows][n][D]
   const float* lse_parts;  // [rows][n]
   int rows, n, D;
-  int rows_per_b;          // rows are (b, h) with h < rows_per_b
+  int rows_per_b;          // rows are (b, r) with r < rows_per_b, r = token * heads + h
+  int heads;
   __nv_bfloat16* o;
-  int64_t o_sb, o_sh;      // element strides of the output rows (b, h)
+  int64_t o_sb, o_st, o_sh;  // element strides of the output rows (b, token, h)
   float* lse;              // [rows] or nullptr
 };
 
@@ -318,8 +319,9 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const CombineArgs a) {
       }
     }
   }
-  const int b = row / a.rows_per_b, h = row % a.rows_per_b;
-  __nv_bfloat16* dst = a.o + (int64_t)b * a.o_sb + (int64_t)h * a.o_sh + lane * V;
+  const int b = row / a.rows_per_b, r = row % a.rows_per_b;
+  const int tok = r / a.heads, h = r % a.heads;
+  __nv_bfloat16* dst = a.o + (int64_t)b * a.o_sb + (int64_t)tok * a.o_st + (int64_t)h * a.o_sh + lane * V;
   if constexpr (V == 4) {
     __nv_bfloat162 p0 = __floats2bfloat162_rn(acc[0], acc[1]);
     __nv_bfloat162 p1 = __floats2bfloat162_rn(acc[2], acc[3]);

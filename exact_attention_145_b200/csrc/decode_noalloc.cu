@@ -106,7 +106,7 @@ extern "C" attn_status attn_decode_noalloc(const attn_decode_params* p, void* st
   if (!p) return ATTN_ERR_INVALID_ARG;
   if (p->B == 0) return attn_decode(p, nullptr, 0, stream);
   const int splits = attn_decode_num_splits(p->B, p->Hq, p->Hkv, p->max_seqlen, p->num_splits);
-  const size_t need = attn_decode_workspace_bytes(p->B, p->Hq, p->D, splits);
+  const size_t need = attn_decode_workspace_bytes(p->B, p->Hq * (p->q_len > 1 ? p->q_len : 1), p->D, splits);
   if (need > static_cast<size_t>(ATTN_DECODE_NOALLOC_MAX_BYTES)) return ATTN_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (attn_status st = scratch_address(&scratch)) return st;

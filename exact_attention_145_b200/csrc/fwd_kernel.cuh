@@ -100,11 +100,16 @@ struct FwdArgs {
   int n_row_units; // prefill: number of row-tile units per (b, head unit)
   int n_units;     // work units in total; the persistent CTAs walk them
   // decode
-  const int32_t* block_table;
+  const int32_t* block_table;  // null: contiguous cache, rows cache_batch_idx[b] (or b)
+  const int32_t* cache_batch_idx;
   int bt_stride;
   const int32_t* seqlens;
   int page_size, num_pages, box_rows, n_splits, tiles_per_split;
   int max_seqlen;   // upper bound on cache_seqlens[b]; larger lengths are clamped and reported
+  // Decode rows: q_len new tokens per sequence x g heads (row r: token r / g,
+  // head r % g of the group); with q_causal token i sees the keys below
+  // seqlen - (q_len - 1 - i). q_bytes: bytes one Q load brings.
+  int q_len, q_causal, q_bytes;
   float* part_o;    // [B][Hq][n_splits][D]
   float* part_lse;  // [B][Hq][n_splits]
   int* status;
@@ -259,7 +264,7 @@ __device__ __forceinline__ int tile_class(const FwdArgs& a, const Work& w, int s
   if constexpr (DECODE) {
     (void)s;
     if (t < w.t_begin || t >= w.t_end) return 0;
-    return (t + 1) * kKeys <= w.seqlen ? 2 : 1;
+    return (t + 1) * kKeys <= w.seqlen - (a.q_causal ? a.q_len - 1 : 0) ? 2 : 1;
   } else {
     const int r0 = w_row0(w, s);
     if (r0 >= a.Sq || t < 0 || t >= a.nK) return 0;
@@ -411,7 +416,9 @@ __device__ __forceinline__ void load_kv_tile(const FwdArgs& a, const Work& w, co
       const int slot = tok % a.page_size;
       int phys = a.num_pages;  // out of range -> TMA fills zeros, no memory read
       if (!absent && tok < w.seqlen && lp < a.bt_stride) {
-        const int pg = a.block_table[(int64_t)w.b * a.bt_stride + lp];
+        // contiguous cache (no block table): one "page" per cache row
+        const int pg = a.block_table ? a.block_table[(int64_t)w.b * a.bt_stride + lp]
+                                     : (a.cache_batch_idx ? a.cache_batch_idx[w.b] : w.b);
         if (pg >= 0 && pg < a.num_pages) {
           phys = pg;
         } else if (a.status && report) {
@@ -520,8 +527,10 @@ __device__ __forceinline__ void mod_chunk(const FwdArgs& a, const Work& w, int s
       for (int i = 0; i < 32; ++i) x[i] = cl * (1.0f - 2.0f * rcp(ex2(x[i] * k2) + 1.0f));
     }
   } else if constexpr (MOD == MOD_ALIBI) {
-    const long q_pos = DECODE ? (long)w.seqlen - 1 : (long)(w_row0(w, s) + row) + a.q_offset;
-    const int head = w_head(w, s) + (DECODE ? row : 0);
+    // decode rows sit at the last q_len positions of the sequence
+    const long q_pos = DECODE ? (long)w.seqlen - a.q_len + min(row / a.g, a.q_len - 1)
+                              : (long)(w_row0(w, s) + row) + a.q_offset;
+    const int head = w_head(w, s) + (DECODE ? row % a.g : 0);
     const float slope = a.alibi[(int64_t)w.b * a.alibi_bstride + min(head, a.Hq - 1)] * kLog2e;
     const float base = slope * (float)((long)t * kKeys + 32 * c - q_pos);
     const float2 SC = make_float2(a.scale_log2, a.scale_log2), SL = make_float2(slope, slope);
@@ -558,7 +567,7 @@ __device__ __forceinline__ MaskRow mask_row(const FwdArgs& a, const Work& w, int
   m.by_id = false;
   if constexpr (DECODE) {
     lo = 0;
-    hi = (long)w.seqlen - 1;
+    hi = (long)w.seqlen - 1 - (a.q_causal ? (long)(a.q_len - 1 - min(row / a.g, a.q_len - 1)) : 0l);
   } else {
     const int qrow = w_row0(w, s) + row;
     const long q_pos = (long)qrow + a.q_offset;
@@ -1161,9 +1170,10 @@ __device__ __forceinline__ bool epilogue(const FwdArgs& a, const CUtensorMap* ma
       const float Lsum = st.l * a0 + l1v * a1;
       const float inv = Lsum > 0.f ? 1.0f / Lsum : 0.f;
       const float w0 = a0 * inv, w1 = a1 * inv;
-      const int h = w.head0 + row;
-      const bool valid = row < a.g;
-      const int64_t prow = ((int64_t)w.b * a.Hq + h) * a.n_splits + w.split;
+      const int h = w.head0 + row % a.g;
+      const int ti = row / a.g;  // new token of the row
+      const bool valid = row < a.g * a.q_len;
+      const int64_t prow = (((int64_t)w.b * a.q_len + ti) * a.Hq + h) * a.n_splits + w.split;
       const uint32_t tO1 = lane_base + 256 + L::kOCols;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
@@ -1328,13 +1338,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ATTN_TRACE_REC(TR_TMA, EV_Q_LOAD, qcnt);
       if (elect_one_sync()) {
-        mbar_arrive_expect_tx(&bar.q_full, L::kNQ * L::kTileBytes);
+        mbar_arrive_expect_tx(&bar.q_full, DECODE ? (uint32_t)a.q_bytes : (uint32_t)(L::kNQ * L::kTileBytes));
         for (int s = 0; s < L::kNQ; ++s)
           for (int c = 0; c < D / 64; ++c) {
             uint8_t* dst = smem + L::kQOff + s * L::kTileBytes + c * L::kChunk;
-            if constexpr (DECODE)
-              tma_load_3d(dst, &map_q, &bar.q_full, c * 64, w.head0, w.b);
-            else
+            if constexpr (DECODE) {
+              // several new tokens: a (64, g, 1, tokens) box puts token i's
+              // heads at rows i*g .. i*g + g - 1
+              if (a.q_len > 1)
+                tma_load_5d(dst, &map_q, &bar.q_full, c * 64, 0, w.hk, 0, w.b);
+              else
+                tma_load_3d(dst, &map_q, &bar.q_full, c * 64, w.head0, w.b);
+            } else
               tma_load_4d(dst, &map_q, &bar.q_full, c * 64, w_row0(w, s), w_head(w, s), w.b);
           }
       }

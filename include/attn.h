@@ -185,6 +185,20 @@ typedef struct {
   int64_t o_stride[2];
   float *lse;                 /* fp32 [B][Hq] contiguous (output); may be NULL */
   int *status;                /* optional device int, ATTN_DEV_* bits */
+  /* Several new tokens per sequence (flash_attn_with_kvcache with q of
+   * seqlen > 1): q and o are [B][q_len][Hq][D], token i at q_token_stride /
+   * o_token_stride elements from token 0; lse is [B][q_len][Hq] contiguous.
+   * The q_len tokens of a sequence sit at its last q_len key positions, and
+   * their q_len x g heads share one 128-row MMA tile: q_len * (Hq / Hkv)
+   * <= 128. 0 means 1 (the fields above alone describe the call). */
+  int q_len;
+  int64_t q_token_stride, o_token_stride;
+  int causal;                 /* q_len > 1: token i sees the first cache_seqlens[b] - (q_len - 1 - i) keys */
+  /* block_table == NULL selects a contiguous cache: k_cache / v_cache are
+   * [num_pages = cache rows][page_size = positions][Hkv][D] and sequence b
+   * reads row cache_batch_idx[b] (row b when cache_batch_idx is NULL);
+   * page_size >= max_seqlen, no divisibility rule. */
+  const int32_t *cache_batch_idx;
 } attn_decode_params;
 
 /* Number of splits attn_decode uses for these sizes (resolves num_splits = 0).
@@ -195,7 +209,7 @@ typedef struct {
 int attn_decode_num_splits(int B, int Hq, int Hkv, int max_seqlen, int num_splits);
 
 /* Workspace bytes attn_decode needs: one fp32 partial O row and LSE per
- * (sequence, query head, split). */
+ * (sequence, query head, split); with q_len new tokens pass Hq * q_len. */
 size_t attn_decode_workspace_bytes(int B, int Hq, int D, int num_splits);
 
 /* Split-KV decode over a paged KV cache (flash_attn_with_kvcache with
@@ -235,6 +249,47 @@ attn_status attn_lse_combine(const float *o_parts, const float *lse_parts, int r
  *  - Allocates and frees nothing. */
 #define ATTN_DECODE_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
 attn_status attn_decode_noalloc(const attn_decode_params *p, void *stream);
+
+/* In-place kv-cache update with rotary embedding (FlashAttention overview,
+ * "Examples": flash_attn_with_kvcache's k, v, rotary_cos, rotary_sin,
+ * rotary_interleaved, cache_batch_idx and block_table arguments). For every
+ * sequence b and new token i (position p = cache_seqlens[b] + i):
+ *   - k_new[b][i] rotated by the angles at p and v_new[b][i] are written to
+ *     the cache at position p (paged: page block_table[b][p / page_size], row
+ *     p % page_size; contiguous: row cache_batch_idx[b] or b, position p);
+ *   - q[b][i] rotated at p is written to q_out (q_out may equal q);
+ *   - seqlens_out[b] = cache_seqlens[b] + Snew when seqlens_out is given.
+ * Rotation: pair j of a head vector is (x[2j], x[2j+1]) when interleaved,
+ * else (x[j], x[j + rotary_dim / 2]), turned by cos/sin[p][j] in fp32 and
+ * rounded to bf16; dims past rotary_dim are copied. rotary_cos == NULL
+ * skips rotation (q_out then receives a copy of q, if both are given).
+ * Kernel-detected errors, OR-ed into *status, skip the row: a page id
+ * outside [0, num_pages) or a logical page past block_table_stride
+ * (ATTN_DEV_BAD_PAGE), a position past the cache or the rotary table
+ * (ATTN_DEV_BAD_LEN). One HBM-bound kernel; nothing is allocated. */
+typedef struct {
+  const void *q;                  /* bf16 [B][Snew][Hq][D] via q_stride, or NULL */
+  int64_t q_stride[3];
+  void *q_out;                    /* bf16, shaped like q, via q_out_stride */
+  int64_t q_out_stride[3];
+  const void *k_new, *v_new;      /* bf16 [B][Snew][Hkv][D] via the strides, or both NULL */
+  int64_t k_new_stride[3], v_new_stride[3];
+  void *k_cache, *v_cache;        /* bf16, same layout: paged [pages][page_size][Hkv][D] or contiguous */
+  int64_t cache_stride[3];        /* element strides of page (row), slot (position), head */
+  const int32_t *block_table;     /* int32 [B][block_table_stride], or NULL for a contiguous cache */
+  int block_table_stride;
+  const int32_t *cache_batch_idx; /* contiguous cache: int32 [B] cache row of each sequence, or NULL */
+  const int32_t *cache_seqlens;   /* int32 [B]: tokens in the cache before the update */
+  int32_t *seqlens_out;           /* int32 [B] or NULL */
+  int B, Snew, Hq, Hkv, D, page_size, num_pages;
+  const float *rotary_cos, *rotary_sin; /* fp32 [rotary_positions][rotary_dim / 2], or NULL */
+  int rotary_dim;                 /* multiple of 16, <= D */
+  int rotary_positions;
+  int rotary_interleaved;
+  int *status;                    /* optional device int */
+} attn_kvcache_update_params;
+
+attn_status attn_kvcache_update(const attn_kvcache_update_params *p, void *stream);
 
 /* Backward of attn_fwd (FlashAttention overview, "Examples": the backward
  * pass of flash_attn_func and its `deterministic` option): dQ, dK, dV for the

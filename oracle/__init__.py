@@ -290,8 +290,10 @@ def _f64_args(q, k, v, dout, scale, mask, window, q_offset, doc_id, mod, softcap
 
 def attn_f64(q, k, v, *, scale: Optional[float] = None, mask: int = MASK_NONE, window=(-1, -1),
              q_offset: int = 0, doc_id=None, mod: int = MOD_NONE, softcap: float = 0.0, alibi=None):
-    """The forward on float64 inputs [B, S, H, D] (no bf16 rounding), for
-    finite-difference checks of the backward. Returns (O [B, Sq, Hq, D], LSE [B, Hq, Sq])."""
+    """The forward on float64 inputs [B, S, H, D] (no bf16 rounding): for
+    finite-difference checks of the backward, and as the reference where the
+    inputs are computed values (a rotated q, gathered cache rows).
+    Returns (O [B, Sq, Hq, D], LSE [B, Hq, Sq])."""
     lib = _load()
     keep = []
     a = _f64_args(q, k, v, None, scale, mask, window, q_offset, doc_id, mod, softcap, alibi, keep)

@@ -172,7 +172,11 @@ def test_decode_argument_checks(lib):
     assert lib.attn_decode(ctypes.byref(p), None, 0, None) == _lib.ATTN_ERR_UNSUPPORTED  # group of 256 heads
     p.Hq = 8
     p.page_size = 48
+    p.block_table = 1 << 20  # the page-size rule binds paged caches only
     assert lib.attn_decode(ctypes.byref(p), None, 0, None) == _lib.ATTN_ERR_UNSUPPORTED
+    p.q_len, p.Hq = 33, 32   # 33 tokens x a group of 4 heads > 128 MMA rows
+    assert lib.attn_decode(ctypes.byref(p), None, 0, None) == _lib.ATTN_ERR_UNSUPPORTED
+    p.q_len, p.Hq = 0, 8
     p.page_size = 256
     assert lib.attn_decode(ctypes.byref(p), None, 0, None) == _lib.ATTN_ERR_INVALID_ARG  # null pointers
     assert lib.attn_lse_combine(None, None, 4, 0, 128, None, 128, None, None) == _lib.ATTN_ERR_INVALID_ARG
