@@ -30,7 +30,7 @@ _lock = threading.Lock()
 _lib = None
 
 MASK_NONE, MASK_CAUSAL, MASK_WINDOW, MASK_DOCUMENT = 0, 1, 2, 3
-MOD_NONE, MOD_SOFTCAP, MOD_ALIBI = 0, 1, 2
+MOD_NONE, MOD_SOFTCAP, MOD_ALIBI, MOD_RELU = 0, 1, 2, 3
 
 
 def build(force: bool = False) -> str:

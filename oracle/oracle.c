@@ -28,7 +28,12 @@
  *   - query i sits at position i + q_offset for the causal / window masks;
  *   - window (left, right), -1 = unbounded: allowed iff
  *       q_pos - kv <= left and kv - q_pos <= right;
- *   - document mask: allowed iff doc[q] == doc[kv] and kv <= q.
+ *   - document mask: allowed iff doc[q] == doc[kv] and kv <= q;
+ *   - ReLU activation wrapper (the talk's example of undoing the softmax
+ *     normalisation and applying a pointwise activation instead):
+ *     O = sum over allowed keys of max(scale * q.k, 0) * v, unnormalised,
+ *     and the LSE slot holds ln of the summed weights (-inf when they sum
+ *     to 0 or no key is allowed).
  */
 #include <math.h>
 #include <pthread.h>
@@ -37,7 +42,7 @@
 #include <string.h>
 
 enum { O_MASK_NONE = 0, O_MASK_CAUSAL = 1, O_MASK_WINDOW = 2, O_MASK_DOCUMENT = 3 };
-enum { O_MOD_NONE = 0, O_MOD_SOFTCAP = 1, O_MOD_ALIBI = 2 };
+enum { O_MOD_NONE = 0, O_MOD_SOFTCAP = 1, O_MOD_ALIBI = 2, O_MOD_RELU = 3 };
 
 static double widen_bf16(uint16_t bits) {
   uint32_t u = (uint32_t)bits << 16;
@@ -111,6 +116,17 @@ static void attn_row(const oracle_attn_args *a, int b, int h, int i, double *o, 
   for (int d = 0; d < a->D; ++d) o[d] = 0.0;
   if (!any) {
     *lse = -INFINITY;
+    return;
+  }
+  if (a->mod == O_MOD_RELU) {
+    double w = 0.0;
+    for (int j = a->kv_begin; j < a->kv_end; ++j) {
+      if (s[j] == -INFINITY || !(s[j] > 0.0)) continue;
+      w += s[j];
+      const uint16_t *vr = a->v + b * a->v_sb + (int64_t)j * a->v_ss + (int64_t)hk * a->v_sh;
+      for (int d = 0; d < a->D; ++d) o[d] += s[j] * widen_bf16(vr[d]);
+    }
+    *lse = w > 0.0 ? log(w) : -INFINITY;
     return;
   }
   double l = 0.0;

@@ -469,3 +469,38 @@ def test_doc_lengths_and_page_permutation():
     assert sum(lens) == 16384 and all(128 <= L <= 2048 for L in lens[:-1]) and 1 <= lens[-1] <= 2048
     perm = W.page_permutation(77, 4096)
     assert sorted(perm.tolist()) == list(range(4096)) and not np.array_equal(perm, np.arange(4096))
+
+
+# ---------------------------------------------------------------- ReLU activation wrapper
+# The talk's activation wrapper (FlexAttention + FlashAttention-4, "activation
+# wrapper ... a ReLU"): O = sum_j max(scale q.k_j, 0) v_j over allowed keys,
+# unnormalised; the LSE slot holds ln of the summed weights.
+
+def test_relu_activation_one_key_and_all_negative():
+    q = bf16(np.array([1.0, 0.0, 0.0, 0.0]).reshape(1, 1, 1, 4))
+    k = bf16(np.array([[2.0, 0.0, 0.0, 0.0], [-4.0, 0.0, 0.0, 0.0]]).reshape(1, 2, 1, 4))
+    v = bf16(np.array([[3.0, -1.0, 0.5, 2.0], [7.0, 7.0, 7.0, 7.0]]).reshape(1, 2, 1, 4))
+    o, lse = oracle.attn(q, k, v, scale=0.5, mod=oracle.MOD_RELU)
+    # weights: relu(0.5 * 2) = 1 for key 0, relu(0.5 * -4) = 0 for key 1
+    assert np.array_equal(o.ravel(), [3.0, -1.0, 0.5, 2.0]) and lse.ravel()[0] == 0.0
+    o, lse = oracle.attn(q, k[:, 1:], v[:, 1:], scale=0.5, mod=oracle.MOD_RELU)
+    assert np.array_equal(o.ravel(), np.zeros(4)) and lse.ravel()[0] == -np.inf
+
+
+def test_relu_activation_homogeneity_linearity_and_mask():
+    q, k, v = rand_qkv(61, 1, 40, 4, 2, 32)
+    o1, l1 = oracle.attn(q, k, v, mod=oracle.MOD_RELU)
+    # doubling q (exact in bf16) doubles every weight: O doubles, LSE gains ln 2
+    o2, l2 = oracle.attn(bf16(2.0 * f64(q)), k, v, mod=oracle.MOD_RELU)
+    assert np.allclose(o2, 2.0 * o1, rtol=1e-12, atol=1e-12)
+    fin = np.isfinite(l1)
+    assert np.allclose(l2[fin], l1[fin] + math.log(2.0), atol=1e-12)
+    # doubling v doubles O and leaves the weights
+    o3, l3 = oracle.attn(q, k, bf16(2.0 * f64(v)), mod=oracle.MOD_RELU)
+    assert np.allclose(o3, 2.0 * o1, rtol=1e-12, atol=1e-12) and np.array_equal(l3, l1)
+    # causal: row 0 sees key 0 only
+    oc, lc = oracle.attn(q, k, v, mod=oracle.MOD_RELU, mask=oracle.MASK_CAUSAL, window=(-1, 0))
+    s00 = max(float(np.dot(f64(q)[0, 0, 0], f64(k)[0, 0, 0])) / math.sqrt(32), 0.0)
+    assert np.allclose(oc[0, 0, 0], s00 * f64(v)[0, 0, 0], atol=1e-12)
+    # a row's output is the row's positive-weighted sum whatever the other rows hold
+    assert np.all(np.isfinite(oc))
