@@ -295,6 +295,45 @@ def decode_setup(torch, ea, w: W.Decode, device, seed_shift: int):
     return dict(step=step, bytes=nbytes, flops=4 * w.D * pairs, splits=splits, d=d)
 
 
+def kvcache_setup(torch, ea, device, seed_shift: int, B=32, Hq=32, Hkv=8, D=128, T=4, kv_len=8192, page=256):
+    """flash_attn_with_kvcache step (speculative-decoding shape): rotary on q and
+    on T new keys, append of the new k/v into a paged cache (block table from
+    a page permutation), causal decode of the T tokens over kv_len keys per
+    sequence. Each step appends at the same positions, so steps are identical.
+    Algorithmic bytes: the K and V rows read (kv_len + T per sequence), q, the
+    new k/v written, O out."""
+    seed = 0xA77E0400 + seed_shift
+    pages_per_seq = (kv_len + T + page - 1) // page
+    P = B * pages_per_seq
+    kc = to_dev(W.normal_bf16(seed, (P, page, Hkv, D)), device)
+    vc = to_dev(W.normal_bf16(seed + 1, (P, page, Hkv, D)), device)
+    q = to_dev(W.normal_bf16(seed + 2, (B, T, Hq, D)), device)
+    kn = to_dev(W.normal_bf16(seed + 3, (B, T, Hkv, D)), device)
+    vn = to_dev(W.normal_bf16(seed + 4, (B, T, Hkv, D)), device)
+    bt = torch.from_numpy(W.page_permutation(seed + 5, P).reshape(B, pages_per_seq)).to(device)
+    sl = torch.full((B,), kv_len, dtype=torch.int32, device=device)
+    j = np.arange(D // 2)
+    ang = np.arange(kv_len + T)[:, None] * (10000.0 ** (-2.0 * j / D))[None, :]
+    cos = torch.from_numpy(np.cos(ang).astype(np.float32)).to(device)
+    sin = torch.from_numpy(np.sin(ang).astype(np.float32)).to(device)
+    new_len = torch.empty_like(sl)
+    q_rot = torch.empty_like(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, T, Hq), dtype=torch.float32, device=device)
+    lib = ea.load_library()
+    splits = lib.attn_decode_num_splits(B, Hq, Hkv, kv_len + T, 0)
+    ws = torch.empty(lib.attn_decode_workspace_bytes(B, Hq * T, D, splits), dtype=torch.uint8, device=device)
+
+    def step(i):
+        ea.attn_kvcache_update(kc, vc, sl, q=q, q_out=q_rot, k=kn, v=vn, block_table=bt, rotary_cos=cos,
+                               rotary_sin=sin, rotary_interleaved=False, seqlens_out=new_len)
+        ea.attn_decode(q_rot, kc, vc, bt, new_len, max_seqlen=kv_len + T, out=o, lse=lse, workspace=ws, causal=True)
+
+    nbytes = 2 * B * (kv_len + T) * Hkv * D * 2 + 2 * (2 * B * T * Hq * D) + 2 * (2 * B * T * Hkv * D)
+    return dict(step=step, bytes=nbytes, splits=splits,
+                name="with_kvcache_gqa_b%d_q%d_kv%d" % (B, T, kv_len))
+
+
 def e2e_prefill(torch, ea, w: W.Prefill, setup, device, steps: int):
     """Same metric through the public API with host buffers: per step, pinned
     host -> device copies of Q, K, V, the forward, device -> host copies of O, LSE."""
@@ -690,6 +729,14 @@ def secondary(torch, ea, device, stream, peaks, rank, barrier, max_over_ranks, w
                    "splits": s["splits"], "roofline_frac": gbs / float(peaks["hbm_gbs"]),
                    "tflops": s["flops"] / (t / steps) / 1e12}
     launches += 2 * steps
+    s = kvcache_setup(torch, ea, device, rank_seed_shift(rank))
+    t, _ = graph_time(torch, s["step"], steps, stream, 5, barrier)
+    t = max_over_ranks(t)
+    gbs = s["bytes"] / (t / steps) / 1e9
+    out[s["name"]] = {"value": gbs * world, "unit": "GB/s", "ms_per_step": 1e3 * t / steps, "bytes": s["bytes"],
+                      "splits": s["splits"], "roofline_frac": gbs / float(peaks["hbm_gbs"]),
+                      "kernels": "kvcache_update_kernel, attn_fwd_kernel<decode>, lse_combine_kernel"}
+    launches += 3 * steps
     out["_launches"] = launches
     return out
 

@@ -23,9 +23,9 @@ from typing import Optional, Tuple
 from . import _lib
 from ._lib import (ATTN_DEV_BAD_LEN, ATTN_DEV_BAD_MASK, ATTN_DEV_BAD_PAGE, ATTN_DEV_TIMEOUT, MASK_CAUSAL,
                    MASK_DOCUMENT, MASK_NONE, MASK_WINDOW,
-                   MOD_ALIBI, MOD_NONE, MOD_SOFTCAP, AttnError)
+                   MOD_ALIBI, MOD_NONE, MOD_RELU, MOD_SOFTCAP, AttnError)
 
-__all__ = ["attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_kvcache_update", "attn_with_kvcache", "attn_decode", "attn_decode_noalloc", "attn_build_block_mask", "attn_lse_combine",
+__all__ = ["attn_fwd", "attn_fwd_qkvpacked", "attn_bwd", "attn_bwd_workspace_bytes", "attn_kvcache_update", "attn_with_kvcache", "attn_decode", "attn_decode_noalloc", "attn_build_block_mask", "attn_lse_combine",
            "BlockMask", "AttnError",
            "load_library", "ATTN_DEV_TIMEOUT", "ATTN_DEV_BAD_PAGE", "ATTN_DEV_BAD_LEN",
            "ATTN_DEV_BAD_MASK"]
@@ -181,10 +181,14 @@ def attn_build_block_mask(Sq: int, Skv: int, *, causal: bool = False, window=Non
     return bm
 
 
-def _mod_args(softcap, alibi_slopes, Hq):
+def _mod_args(softcap, alibi_slopes, Hq, activation=None):
     torch = _torch()
-    if softcap is not None and alibi_slopes is not None:
-        raise ValueError("choose one score mod: softcap or alibi_slopes")
+    if sum(x is not None for x in (softcap, alibi_slopes, activation)) > 1:
+        raise ValueError("choose one score mod: softcap, alibi_slopes or activation")
+    if activation is not None:
+        if activation != "relu":
+            raise ValueError("activation must be 'relu'")
+        return MOD_RELU, 0.0, None, 0
     if softcap is not None:
         return MOD_SOFTCAP, float(softcap), None, 0
     if alibi_slopes is not None:
@@ -197,10 +201,13 @@ def _mod_args(softcap, alibi_slopes, Hq):
 
 def attn_fwd(q, k, v, *, scale: Optional[float] = None, causal: bool = False, window=None, q_offset: int = 0,
              doc_id=None, block_mask: Optional[BlockMask] = None, softcap: Optional[float] = None,
-             alibi_slopes=None, out=None, lse=None, status=None, with_lse: bool = True, stream=None):
+             alibi_slopes=None, activation: Optional[str] = None, out=None, lse=None, status=None,
+             with_lse: bool = True, stream=None):
     """Exact attention forward. q [B, Sq, Hq, D], k/v [B, Skv, Hkv, D] bf16 (any
     strides with a contiguous last dim, e.g. BHSD views). Returns (O, LSE):
-    O bf16 [B, Sq, Hq, D] and LSE fp32 [B, Hq, Sq] (natural log)."""
+    O bf16 [B, Sq, Hq, D] and LSE fp32 [B, Hq, Sq] (natural log).
+    activation="relu" replaces the softmax by the activation wrapper:
+    O = sum_j max(scale q.k_j, 0) v_j over allowed keys, LSE = ln of the weights' sum."""
     torch = _torch()
     _check_bf16("q", q, 4)
     _check_bf16("k", k, 4)
@@ -225,11 +232,31 @@ def attn_fwd(q, k, v, *, scale: Optional[float] = None, causal: bool = False, wi
     if kind == MASK_DOCUMENT and block_mask is None:
         block_mask = attn_build_block_mask(Sq, Skv, doc_id=doc_id, stream=stream)
     p.block_mask = ctypes.pointer(block_mask.c) if block_mask is not None else None
-    p.mod, p.softcap, p.alibi_slopes, p.alibi_batch_stride = _mod_args(softcap, alibi_slopes, Hq)
+    p.mod, p.softcap, p.alibi_slopes, p.alibi_batch_stride = _mod_args(softcap, alibi_slopes, Hq, activation)
     p.status = _ptr(status)
     h = _stream_handle(q.device) if stream is None else stream
     _lib.check(_lib.load().attn_fwd(ctypes.byref(p), h), "attn_fwd")
     return out, lse
+
+
+def attn_fwd_qkvpacked(qkv, *, num_heads_q: Optional[int] = None, **kw):
+    """QKV-packed entry (flash_attn_qkvpacked_func, FlashAttention overview):
+    qkv bf16 [B, S, 3, H, D] (Q, K, V of H heads each), or [B, S, Hq + 2 Hkv, D]
+    with num_heads_q = Hq for packed GQA (the Q heads, then K, then V). The
+    three operands are strided views of the one buffer, read in place by
+    attn_fwd's tensor maps; keyword arguments are attn_fwd's."""
+    if qkv.dim() == 5:
+        if qkv.shape[2] != 3:
+            raise ValueError("qkv [B, S, 3, H, D] expected")
+        return attn_fwd(qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2], **kw)
+    if qkv.dim() != 4 or num_heads_q is None:
+        raise ValueError("qkv [B, S, 3, H, D], or [B, S, Hq + 2 Hkv, D] with num_heads_q")
+    Hq = int(num_heads_q)
+    rest = qkv.shape[2] - Hq
+    if rest <= 0 or rest % 2 != 0:
+        raise ValueError("the packed head count must be num_heads_q + 2 Hkv")
+    Hkv = rest // 2
+    return attn_fwd(qkv[:, :, :Hq], qkv[:, :, Hq:Hq + Hkv], qkv[:, :, Hq + Hkv:], **kw)
 
 
 def _bwd_params(q, k, v, out, lse, dout, dq, dk, dv, scale, causal, window, q_offset, deterministic, status):

@@ -23,7 +23,7 @@ def lib_path() -> str:
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_WORKSPACE = range(5)
 ATTN_DEV_TIMEOUT, ATTN_DEV_BAD_PAGE, ATTN_DEV_BAD_LEN, ATTN_DEV_BAD_MASK = 1, 2, 4, 8
 MASK_NONE, MASK_CAUSAL, MASK_WINDOW, MASK_DOCUMENT = range(4)
-MOD_NONE, MOD_SOFTCAP, MOD_ALIBI = range(3)
+MOD_NONE, MOD_SOFTCAP, MOD_ALIBI, MOD_RELU = range(4)
 
 EXPORTS = ("attn_block_mask_bytes", "attn_block_mask_layout", "attn_build_block_mask", "attn_fwd",
            "attn_decode_num_splits", "attn_decode_workspace_bytes", "attn_decode", "attn_lse_combine",

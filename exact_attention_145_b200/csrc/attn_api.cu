@@ -120,6 +120,11 @@ attn_status launch_fwd_bm(const CUtensorMap& mq, const CUtensorMap& mk, const CU
       return launch_fwd_mod<D, DECODE, MOD_SOFTCAP, BM>(mq, mk, mv, mo, a, grid, stream);
     case MOD_ALIBI:
       return launch_fwd_mod<D, DECODE, MOD_ALIBI, BM>(mq, mk, mv, mo, a, grid, stream);
+    case MOD_RELU:
+      if constexpr (DECODE)
+        return ATTN_ERR_UNSUPPORTED;
+      else
+        return launch_fwd_mod<D, DECODE, MOD_RELU, BM>(mq, mk, mv, mo, a, grid, stream);
     default:
       return launch_fwd_mod<D, DECODE, MOD_NONE, BM>(mq, mk, mv, mo, a, grid, stream);
   }
@@ -171,7 +176,8 @@ attn_status check_mods(attn_mod_kind mod, float softcap, const float* alibi, int
   if (mod == ATTN_MOD_SOFTCAP && !(softcap > 0.f && std::isfinite(softcap))) return ATTN_ERR_INVALID_ARG;
   if (mod == ATTN_MOD_ALIBI && (alibi == nullptr || (alibi_bstride != 0 && alibi_bstride != Hq)))
     return ATTN_ERR_INVALID_ARG;
-  if (mod != ATTN_MOD_NONE && mod != ATTN_MOD_SOFTCAP && mod != ATTN_MOD_ALIBI) return ATTN_ERR_INVALID_ARG;
+  if (mod != ATTN_MOD_NONE && mod != ATTN_MOD_SOFTCAP && mod != ATTN_MOD_ALIBI && mod != ATTN_MOD_RELU)
+    return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;
 }
 
@@ -754,6 +760,7 @@ attn_status attn_decode(const attn_decode_params* p, void* workspace, size_t wor
   if (!strides_ok(p->q_stride, 2) || !strides_ok(p->cache_stride, 3) || !strides_ok(p->o_stride, 2))
     return ATTN_ERR_UNSUPPORTED;
   if (attn_status st = check_mods(p->mod, p->softcap, p->alibi_slopes, p->alibi_batch_stride, p->Hq)) return st;
+  if (p->mod == ATTN_MOD_RELU) return ATTN_ERR_UNSUPPORTED;  // split partials assume normalised rows
   const int splits = attn_decode_num_splits(p->B, p->Hq, p->Hkv, p->max_seqlen, p->num_splits);
   const size_t need = attn_decode_workspace_bytes(p->B, p->Hq * q_len, p->D, splits);
   if (!workspace || !aligned16(workspace)) return ATTN_ERR_INVALID_ARG;

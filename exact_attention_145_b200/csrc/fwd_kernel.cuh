@@ -71,7 +71,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 enum : int { MASK_NONE = 0, MASK_CAUSAL = 1, MASK_WINDOW = 2, MASK_DOCUMENT = 3 };
-enum : int { MOD_NONE = 0, MOD_SOFTCAP = 1, MOD_ALIBI = 2 };
+enum : int { MOD_NONE = 0, MOD_SOFTCAP = 1, MOD_ALIBI = 2, MOD_RELU = 3 };
 enum : int { DEV_TIMEOUT = 1, DEV_BAD_PAGE = 2, DEV_BAD_LEN = 4, DEV_BAD_MASK = 8 };
 
 struct FwdArgs {
@@ -526,6 +526,15 @@ __device__ __forceinline__ void mod_chunk(const FwdArgs& a, const Work& w, int s
 #pragma unroll
       for (int i = 0; i < 32; ++i) x[i] = cl * (1.0f - 2.0f * rcp(ex2(x[i] * k2) + 1.0f));
     }
+  } else if constexpr (MOD == MOD_RELU) {
+    // activation wrapper: the scaled score itself (the ReLU follows the mask)
+    const float2 SC = make_float2(a.scale, a.scale);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float2 r = mul2(make_float2(x[i], x[i + 1]), SC);
+      x[i] = r.x;
+      x[i + 1] = r.y;
+    }
   } else if constexpr (MOD == MOD_ALIBI) {
     // decode rows sit at the last q_len positions of the sequence
     const long q_pos = DECODE ? (long)w.seqlen - a.q_len + min(row / a.g, a.q_len - 1)
@@ -767,6 +776,44 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
                                              uint64_t* p_ready) {
   float x[kKeys];
   const float NEG_INF = -__int_as_float(0x7f800000);
+  if constexpr (MOD == MOD_RELU) {
+    // Activation wrapper (the FlexAttention talk's ReLU example): P = max(scale
+    // * s, 0) on allowed pairs, no running max, no rescale, no normalisation.
+    // The row keeps m = 0 and l = the summed weights, so the epilogue writes
+    // ln(l) in the LSE slot and O unscaled.
+    float wsum = 0.f;
+    if (cls == 0) {
+      uint32_t pk[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) pk[j] = 0u;
+      tmem_st32(tS, pk);
+      tmem_st32(tS + 32, pk);
+    } else {
+      if (cls == 2)
+        (void)prepare_tile<DECODE, MOD, false, BM>(a, w, s, row, t, tS, x);
+      else
+        (void)prepare_tile<DECODE, MOD, true, BM>(a, w, s, row, t, tS, x);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float p0 = fmaxf(x[32 * c + 2 * j], 0.f), p1 = fmaxf(x[32 * c + 2 * j + 1], 0.f);
+          wsum += p0 + p1;
+          pk[j] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + 16 * c, pk);
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    mbar_arrive(p_ready);
+    st.m = 0.f;
+    st.l += wsum;
+    (void)tO;
+    (void)first;
+    return;
+  }
   const float mult = MOD == MOD_NONE ? a.scale_log2 : 1.0f;  // x * mult is the log2-domain score
   const float2 MULT = make_float2(mult, mult);
   float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
@@ -874,7 +921,7 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
 // the MMAs pays for the extra hand-offs (+6-8 % measured). Without a mod the
 // whole-tile schedule is faster (the half schedule measured 5 % slower).
 template <bool DECODE, int MOD>
-constexpr bool kHalfTiles = !DECODE && MOD != MOD_NONE;
+constexpr bool kHalfTiles = !DECODE && MOD != MOD_NONE && MOD != MOD_RELU;
 
 // With half tiles: P for keys
 // 0-63 goes to S(s) columns [0, 32) and P for keys 64-127 to [64, 96), so:
@@ -1106,7 +1153,8 @@ __device__ __forceinline__ bool epilogue(const FwdArgs& a, const CUtensorMap* ma
     const int qrow = r0 + row;
     const bool valid = qrow < a.Sq && r0 < a.Sq;
     const bool box_valid = r0 + 32 * wq < a.Sq;  // warp-uniform; rows past Sq are clipped by the map
-    const float inv_l = st.l > 0.f ? 1.0f / st.l : 0.f;
+    // the ReLU activation wrapper leaves O unnormalised
+    const float inv_l = a.mod == MOD_RELU ? 1.0f : (st.l > 0.f ? 1.0f / st.l : 0.f);
     uint8_t* stage = extra + (s * 4 + wq) * L::kStageWarpBytes;
     const uint32_t srow = smem_u32(stage) + lane * 128;
 #pragma unroll

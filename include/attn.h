@@ -70,7 +70,12 @@ typedef enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_WINDOW = 2, A
  * (FA4 talk, score_mod hooks; flash_attn alibi_slopes and softcapping):
  *   SOFTCAP   s -> softcap * tanh(s / softcap)
  *   ALIBI     s -> s + slope[b][h] * (j - q_pos)                                */
-typedef enum { ATTN_MOD_NONE = 0, ATTN_MOD_SOFTCAP = 1, ATTN_MOD_ALIBI = 2 } attn_mod_kind;
+/* Score modifiers (FlexAttention score_mod hooks; flash_attn_func's softcap
+ * and alibi_slopes). ATTN_MOD_RELU is the talk's activation wrapper: the
+ * softmax normalisation is undone and each allowed scaled score passes
+ * through ReLU, O = sum_j max(scale q.k_j, 0) v_j, with ln(sum_j of those
+ * weights) in the LSE slot (-inf when they sum to 0); attn_fwd only. */
+typedef enum { ATTN_MOD_NONE = 0, ATTN_MOD_SOFTCAP = 1, ATTN_MOD_ALIBI = 2, ATTN_MOD_RELU = 3 } attn_mod_kind;
 
 typedef struct {
   attn_mask_kind kind;
