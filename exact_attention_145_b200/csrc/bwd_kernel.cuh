@@ -27,6 +27,9 @@
 // Warp roles (320 threads): warps 0-7 compute (warp w: TMEM lanes
 // 32 (w % 4) .. +31 = the tile's rows, columns half w / 4), warp 8 MMA issue
 // (owns TMEM), warp 9 TMA producer. Every wait is bounded (sm100.cuh).
+// Each step runs as two column halves with their own barriers: the tensor
+// pipe computes half B's S / dP while half A's warps compute, then half A's
+// accumulation and the next step's half A products while half B computes.
 #pragma once
 
 #include <cstdint>
@@ -241,7 +244,7 @@ struct BLayout {
   // dq: Q, dO of the unit, then a 2-slot ring of (K, V) per step.
   static constexpr int kFixOff = 0;                   // two unit tiles
   static constexpr int kRingOff = 2 * kTileBytes;     // 2 slots x two step tiles
-  static constexpr int kVecOff = kRingOff + 4 * kTileBytes;  // dkdv: 2 slots x (log2e*LSE, delta) x 128 floats
+  static constexpr int kVecOff = kRingOff + 4 * kTileBytes;  // dkdv: 2 slots x 2 halves x (log2e*LSE, delta) x 64 floats
   static constexpr int kBarOff = kVecOff + 2 * 2 * kTile * 4;
   // Each CTA allocates all 512 TMEM columns, so two CTAs must never share an
   // SM: the request is padded past half of the SM's 228 KB of shared memory.
@@ -254,11 +257,11 @@ struct BLayout {
 struct BBarriers {
   uint64_t fix_full, fix_empty;  // unit tiles loaded / released
   uint64_t ring_full[2], ring_empty[2];
-  uint64_t mm1_ready;   // the step's first two products (S / dP) are in TMEM
-  uint64_t comp_ready;  // the compute warps wrote P^T / dS^T (dkdv) or dS (dq): 256 arrivals
-  uint64_t acc_done;    // the unit's accumulators are final
-  uint64_t acc_free;    // the epilogue read them: 256 arrivals
-  uint64_t vec_ready[2];  // dkdv: the step's LSE / delta columns are in shared memory (256 arrivals)
+  uint64_t mm1_ready[2];   // per column half: the step's S / dP products are in TMEM
+  uint64_t comp_ready[2];  // per half: its warps wrote P^T / dS^T (dkdv) or dS (dq): 128 arrivals
+  uint64_t acc_done;       // the unit's accumulators are final
+  uint64_t acc_free;       // the epilogue read them: 256 arrivals
+  uint64_t vec_ready[2][2];  // dkdv, [slot][half]: the half's LSE / delta columns are in shared memory
   uint64_t final_mma;
   uint32_t tmem_base;
   int abort_flag;
@@ -316,7 +319,8 @@ __device__ __forceinline__ float bex2(float x) {
 
 // ---------------------------------------------------------------- dK / dV
 // TMEM columns: S^T [0, 128), dP^T [128, 256), dV [256, 256 + D), dK [256 + D, 256 + 2D).
-// MMA order per step: S^T, dP^T | (compute) | dV, dK, S^T(next), dP^T(next).
+// MMA order per step, by 64-query halves A / B: S^T_A dP^T_A S^T_B dP^T_B |
+// (compute A) | dV_A dK_A S^T_A(next) dP^T_A(next) | (compute B) | dV_B dK_B ...
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -336,12 +340,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bar.ring_full[i], 1);
       mbar_init(&bar.ring_empty[i], 1);
     }
-    mbar_init(&bar.mm1_ready, 1);
-    mbar_init(&bar.comp_ready, kBCompute);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bar.mm1_ready[h], 1);
+      mbar_init(&bar.comp_ready[h], kTile);
+      mbar_init(&bar.vec_ready[0][h], kTile);
+      mbar_init(&bar.vec_ready[1][h], kTile);
+    }
     mbar_init(&bar.acc_done, 1);
     mbar_init(&bar.acc_free, kBCompute);
-    mbar_init(&bar.vec_ready[0], kBCompute);
-    mbar_init(&bar.vec_ready[1], kBCompute);
     mbar_init(&bar.final_mma, 1);
     fence_barrier_init();
   }
@@ -413,27 +419,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     constexpr uint32_t kHi = sdesc_sw128_hi(1024);
-    constexpr uint32_t idesc_mm1 = idesc_bf16_f32(128, 128, 0, 0);  // K-major A and B
-    constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);    // B MN-major (rows x D tiles)
+    constexpr uint32_t idesc_mm1 = idesc_bf16_f32(128, 64, 0, 0);  // K-major A and B, one 64-query half
+    constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);   // B MN-major (rows x D tiles)
     constexpr uint32_t kTileUnits = L::kTileBytes >> 4;
+    constexpr uint32_t kHalfRows = (64 * 128) >> 4;                  // 64 rows of a SW128 chunk
     const uint32_t k_lo = sdesc_sw128_lo(smem_u32(smem + L::kFixOff), 16);
     const uint32_t v_lo = k_lo + kTileUnits;
     const uint32_t ring_lo = sdesc_sw128_lo(smem_u32(smem + L::kRingOff), 16);
     const uint32_t ring_mn = sdesc_sw128_lo(smem_u32(smem + L::kRingOff), L::kChunk);
-    // S^T = K Q^T into [0, 128) and dP^T = V dO^T into [128, 256) for ring slot `slot`.
-    auto mm1 = [&](int slot) {
-      const uint32_t qa = ring_lo + (uint32_t)slot * 2 * kTileUnits, da = qa + kTileUnits;
+    // Half h of the step in ring slot `slot`: S^T = K Q^T for queries 64h..64h+63
+    // into columns [64h, 64h + 64), dP^T = V dO^T into [128 + 64h, ...).
+    auto mm1_half = [&](int slot, int h) {
+      const uint32_t qa = ring_lo + (uint32_t)slot * 2 * kTileUnits + (uint32_t)h * kHalfRows, da = qa + kTileUnits;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
-        mma_ss(tmem, sdesc_join(k_lo + off, kHi), sdesc_join(qa + off, kHi), idesc_mm1, kk > 0);
+        mma_ss(tmem + 64 * h, sdesc_join(k_lo + off, kHi), sdesc_join(qa + off, kHi), idesc_mm1, kk > 0);
       }
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
-        mma_ss(tmem + 128, sdesc_join(v_lo + off, kHi), sdesc_join(da + off, kHi), idesc_mm1, kk > 0);
+        mma_ss(tmem + 128 + 64 * h, sdesc_join(v_lo + off, kHi), sdesc_join(da + off, kHi), idesc_mm1, kk > 0);
       }
-      mma_commit(&bar.mm1_ready);
+      mma_commit(&bar.mm1_ready[h]);
+    };
+    // Half h's accumulation: dV += P^T dO and dK += dS^T Q over queries 64h..64h+63.
+    auto acc_half = [&](int slot, int h, bool first) {
+      const uint32_t qmn = ring_mn + (uint32_t)slot * 2 * kTileUnits, dmn = qmn + kTileUnits;
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int kk = 4 * h + k4;
+        mma_ts(tmem + 256, tmem + packed_col(kk), sdesc_join(dmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
+               (!first || kk > 0) ? 1u : 0u);
+      }
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int kk = 4 * h + k4;
+        mma_ts(tmem + 256 + D, tmem + 128 + packed_col(kk), sdesc_join(qmn + ((kk * 16 * 128) >> 4), kHi),
+               idesc_acc, (!first || kk > 0) ? 1u : 0u);
+      }
     };
     int ucnt = 0, gstep = 0;
     bool ok = true;
@@ -445,35 +469,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = wait_all(&bar.fix_full, ucnt & 1) && wait_all(&bar.ring_full[gstep & 1], (gstep >> 1) & 1);
       if (!ok) break;
       tc_fence_after();
-      if (elect_one_sync()) mm1(gstep & 1);
+      if (elect_one_sync()) {
+        mm1_half(gstep & 1, 0);
+        mm1_half(gstep & 1, 1);
+      }
       __syncwarp();
       for (int s = 0; s < w.n; ++s) {
         const int g = gstep + s, slot = g & 1;
         const bool more = s + 1 < w.n;
-        if (more && !wait_all(&bar.ring_full[(g + 1) & 1], ((g + 1) >> 1) & 1)) { ok = false; break; }
-        if (!wait_spin_all(&bar.comp_ready, g & 1)) { ok = false; break; }
+        // half A: its accumulation, then the next step's half A products
+        if (!wait_spin_all(&bar.comp_ready[0], g & 1)) { ok = false; break; }
         // The unit's first accumulation overwrites dV / dK: the previous
         // unit's epilogue must have read them.
         if (s == 0 && ucnt > 0 && !wait_all(&bar.acc_free, (ucnt - 1) & 1)) { ok = false; break; }
+        if (more && !wait_all(&bar.ring_full[(g + 1) & 1], ((g + 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         if (elect_one_sync()) {
-          const uint32_t qmn = ring_mn + (uint32_t)slot * 2 * kTileUnits, dmn = qmn + kTileUnits;
-          // dV += P^T dO: P^T packed in S^T's columns, dO rows 16kk..
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + 256, tmem + packed_col(kk), sdesc_join(dmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
-                   (s > 0 || kk > 0) ? 1u : 0u);
-          // dK += dS^T Q: dS^T packed in dP^T's columns
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + 256 + D, tmem + 128 + packed_col(kk), sdesc_join(qmn + ((kk * 16 * 128) >> 4), kHi),
-                   idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
+          acc_half(slot, 0, s == 0);
+          if (more) mm1_half((g + 1) & 1, 0);
+        }
+        __syncwarp();
+        // half B: its accumulation, the slot's release, the next half B products
+        if (!wait_spin_all(&bar.comp_ready[1], g & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one_sync()) {
+          acc_half(slot, 1, s == 0);
           mma_commit(&bar.ring_empty[slot]);
-          if (!more) {
+          if (more) {
+            mm1_half((g + 1) & 1, 1);
+          } else {
             mma_commit(&bar.acc_done);
             mma_commit(&bar.fix_empty);
-          } else {
-            mm1((g + 1) & 1);
           }
         }
         __syncwarp();
@@ -519,32 +545,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (a.wl >= 0) qhi_i = min(qhi_i, key + a.wl - a.q_offset);
       }
       if (!real) qhi_i = -1;
+      // Column values of a step for this half's 64 queries (log2e * LSE and
+      // delta): thread row fetches LSE (rows 0-63) or delta (rows 64-127) of
+      // query qt*128 + 64 half + row % 64. The global load for step s + 1 is
+      // issued during step s, so its latency is off the per-step chain.
+      auto column_value = [&](int s) -> float {
+        const int qt = w.qlo + (w.s0 + s) / a.g, h = w.hk * a.g + (w.s0 + s) % a.g;
+        const int typ = row / 64, qi = qt * kTile + 64 * half + row % 64;
+        float val = typ == 0 ? POS_INF : 0.f;
+        if (qi < a.Sq) {
+          const int64_t ix = ((int64_t)w.b * a.Hq + h) * a.Sq + qi;
+          if (typ == 0) {
+            const float l = __ldg(a.lse + ix);
+            // LSE -inf (a row with no allowed key): none of its pairs is allowed either
+            val = l == NEG_INF ? POS_INF : l * kLog2eB;
+          } else {
+            val = __ldg(a.delta + ix);
+          }
+        }
+        return val;
+      };
+      float next_val = column_value(0);
       for (int s = 0; s < w.n; ++s) {
         const int g = gstep + s, slot = g & 1;
-        const int qt = w.qlo + (w.s0 + s) / a.g, h = w.hk * a.g + (w.s0 + s) % a.g;
-        // Column values of the step (log2e * LSE and delta of the q tile's
-        // queries): half 0 fetches the LSE of query qt*128 + row, half 1 its
-        // delta, into a shared, double-buffered array; a bounded mbarrier
-        // (256 arrivals) publishes it.
-        float* vec = reinterpret_cast<float*>(smem + L::kVecOff) + slot * 2 * kTile;
-        {
-          const int qi = qt * kTile + row;
-          float val = half == 0 ? POS_INF : 0.f;
-          if (qi < a.Sq) {
-            const int64_t ix = ((int64_t)w.b * a.Hq + h) * a.Sq + qi;
-            if (half == 0) {
-              const float l = a.lse[ix];
-              // LSE -inf (a row with no allowed key): none of its pairs is allowed either
-              val = l == NEG_INF ? POS_INF : l * kLog2eB;
-            } else {
-              val = a.delta[ix];
-            }
-          }
-          vec[half * kTile + row] = val;
-          mbar_arrive(&bar.vec_ready[slot]);
-        }
-        if (!wait_spin_all(&bar.mm1_ready, g & 1)) { ok = false; break; }
-        if (!wait_spin_all(&bar.vec_ready[slot], (g >> 1) & 1)) { ok = false; break; }
+        const int qt = w.qlo + (w.s0 + s) / a.g;
+        // the half's own double-buffered array, published by a bounded
+        // mbarrier (128 arrivals)
+        float* vec = reinterpret_cast<float*>(smem + L::kVecOff) + (slot * 2 + half) * kTile;
+        vec[row] = next_val;
+        mbar_arrive(&bar.vec_ready[slot][half]);
+        if (s + 1 < w.n) next_val = column_value(s + 1);
+        if (!wait_spin_all(&bar.mm1_ready[half], g & 1)) { ok = false; break; }
+        if (!wait_spin_all(&bar.vec_ready[slot][half], (g >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const bool full = pair_full(a, qt, w.t);
 #pragma unroll 1
@@ -557,8 +589,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           reg_fence_f<32>(x);
           reg_fence_f<32>(dp);
           const uint32_t bits = full ? 0xffffffffu : range_bits(qlo_i, qhi_i, (long)qt * kTile + 32 * c);
-          const float4* l2v = reinterpret_cast<const float4*>(vec + 32 * c);
-          const float4* dlv = reinterpret_cast<const float4*>(vec + kTile + 32 * c);
+          const float4* l2v = reinterpret_cast<const float4*>(vec + 32 * cc);
+          const float4* dlv = reinterpret_cast<const float4*>(vec + 64 + 32 * cc);
           uint32_t pk[16], dk[16];
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
@@ -583,7 +615,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bar.comp_ready);
+        mbar_arrive(&bar.comp_ready[half]);
       }
       if (!ok) break;
       // epilogue: dV, dK rows, this thread's half of the columns
@@ -687,7 +719,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dkdv_reduce_kernel(const BwdArgs
 // ---------------------------------------------------------------- dQ
 // TMEM columns: S [0, 128), dP [128, 256), dQ [256, 256 + D). dS (bf16
 // pairs) is packed into S's columns. MMA order per step:
-// S, dP | (compute) | dQ, S(next), dP(next).
+// by 64-key halves: S_A dP_A S_B dP_B | (compute A) | dQ_A S_A(next) dP_A(next) | (compute B) | dQ_B ...
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -707,8 +739,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bar.ring_full[i], 1);
       mbar_init(&bar.ring_empty[i], 1);
     }
-    mbar_init(&bar.mm1_ready, 1);
-    mbar_init(&bar.comp_ready, kBCompute);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bar.mm1_ready[h], 1);
+      mbar_init(&bar.comp_ready[h], kTile);
+    }
     mbar_init(&bar.acc_done, 1);
     mbar_init(&bar.acc_free, kBCompute);
     mbar_init(&bar.final_mma, 1);
@@ -782,27 +816,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     constexpr uint32_t kHi = sdesc_sw128_hi(1024);
-    constexpr uint32_t idesc_mm1 = idesc_bf16_f32(128, 128, 0, 0);
+    constexpr uint32_t idesc_mm1 = idesc_bf16_f32(128, 64, 0, 0);  // one 64-key half
     constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
     constexpr uint32_t kTileUnits = L::kTileBytes >> 4;
+    constexpr uint32_t kHalfRows = (64 * 128) >> 4;
     const uint32_t q_lo = sdesc_sw128_lo(smem_u32(smem + L::kFixOff), 16);
     const uint32_t do_lo = q_lo + kTileUnits;
     const uint32_t ring_lo = sdesc_sw128_lo(smem_u32(smem + L::kRingOff), 16);
     const uint32_t ring_mn = sdesc_sw128_lo(smem_u32(smem + L::kRingOff), L::kChunk);
-    // S = Q K^T into [0, 128) and dP = dO V^T into [128, 256) for ring slot `slot`.
-    auto mm1 = [&](int slot) {
-      const uint32_t ka = ring_lo + (uint32_t)slot * 2 * kTileUnits, va = ka + kTileUnits;
+    // Half h: S = Q K^T for keys 64h..64h+63 into [64h, 64h + 64), dP = dO V^T into [128 + 64h, ...).
+    auto mm1_half = [&](int slot, int h) {
+      const uint32_t ka = ring_lo + (uint32_t)slot * 2 * kTileUnits + (uint32_t)h * kHalfRows, va = ka + kTileUnits;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
-        mma_ss(tmem, sdesc_join(q_lo + off, kHi), sdesc_join(ka + off, kHi), idesc_mm1, kk > 0);
+        mma_ss(tmem + 64 * h, sdesc_join(q_lo + off, kHi), sdesc_join(ka + off, kHi), idesc_mm1, kk > 0);
       }
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = ((kk / 4) * L::kChunk + (kk % 4) * 32) >> 4;
-        mma_ss(tmem + 128, sdesc_join(do_lo + off, kHi), sdesc_join(va + off, kHi), idesc_mm1, kk > 0);
+        mma_ss(tmem + 128 + 64 * h, sdesc_join(do_lo + off, kHi), sdesc_join(va + off, kHi), idesc_mm1, kk > 0);
       }
-      mma_commit(&bar.mm1_ready);
+      mma_commit(&bar.mm1_ready[h]);
+    };
+    // Half h's accumulation: dQ += dS K over keys 64h..64h+63.
+    auto acc_half = [&](int slot, int h, bool first) {
+      const uint32_t kmn = ring_mn + (uint32_t)slot * 2 * kTileUnits;
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int kk = 4 * h + k4;
+        mma_ts(tmem + 256, tmem + packed_col(kk), sdesc_join(kmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
+               (!first || kk > 0) ? 1u : 0u);
+      }
     };
     int ucnt = 0, gstep = 0;
     bool ok = true;
@@ -814,28 +859,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = wait_all(&bar.fix_full, ucnt & 1) && wait_all(&bar.ring_full[gstep & 1], (gstep >> 1) & 1);
       if (!ok) break;
       tc_fence_after();
-      if (elect_one_sync()) mm1(gstep & 1);
+      if (elect_one_sync()) {
+        mm1_half(gstep & 1, 0);
+        mm1_half(gstep & 1, 1);
+      }
       __syncwarp();
       for (int s = 0; s < w.n; ++s) {
         const int g = gstep + s, slot = g & 1;
         const bool more = s + 1 < w.n;
-        if (more && !wait_all(&bar.ring_full[(g + 1) & 1], ((g + 1) >> 1) & 1)) { ok = false; break; }
-        if (!wait_spin_all(&bar.comp_ready, g & 1)) { ok = false; break; }
+        if (!wait_spin_all(&bar.comp_ready[0], g & 1)) { ok = false; break; }
         if (s == 0 && ucnt > 0 && !wait_all(&bar.acc_free, (ucnt - 1) & 1)) { ok = false; break; }
+        if (more && !wait_all(&bar.ring_full[(g + 1) & 1], ((g + 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         if (elect_one_sync()) {
-          const uint32_t kmn = ring_mn + (uint32_t)slot * 2 * kTileUnits;
-          // dQ += dS K: dS packed in S's columns, K rows 16kk..
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tmem + 256, tmem + packed_col(kk), sdesc_join(kmn + ((kk * 16 * 128) >> 4), kHi), idesc_acc,
-                   (s > 0 || kk > 0) ? 1u : 0u);
+          acc_half(slot, 0, s == 0);
+          if (more) mm1_half((g + 1) & 1, 0);
+        }
+        __syncwarp();
+        if (!wait_spin_all(&bar.comp_ready[1], g & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one_sync()) {
+          acc_half(slot, 1, s == 0);
           mma_commit(&bar.ring_empty[slot]);
-          if (!more) {
+          if (more) {
+            mm1_half((g + 1) & 1, 1);
+          } else {
             mma_commit(&bar.acc_done);
             mma_commit(&bar.fix_empty);
-          } else {
-            mm1((g + 1) & 1);
           }
         }
         __syncwarp();
@@ -884,18 +934,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int s = 0; s < w.n; ++s) {
         const int g = gstep + s;
         const int t = w.klo + s;
-        if (!wait_spin_all(&bar.mm1_ready, g & 1)) { ok = false; break; }
+        if (!wait_spin_all(&bar.mm1_ready[half], g & 1)) { ok = false; break; }
         tc_fence_after();
         const bool full = pair_full(a, w.qt, t);
-#pragma unroll 1
+        // both chunks' S and dP columns in one TMEM round trip
+        float xs[2][32], dps[2][32];
+        tmem_ld32f(lane_base + 64 * half, xs[0]);
+        tmem_ld32f(lane_base + 64 * half + 32, xs[1]);
+        tmem_ld32f(lane_base + 128 + 64 * half, dps[0]);
+        tmem_ld32f(lane_base + 128 + 64 * half + 32, dps[1]);
+        tmem_ld_wait();
+        reg_fence_f<32>(xs[0]);
+        reg_fence_f<32>(xs[1]);
+        reg_fence_f<32>(dps[0]);
+        reg_fence_f<32>(dps[1]);
+#pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c = 2 * half + cc;
-          float x[32], dp[32];
-          tmem_ld32f(lane_base + 32 * c, x);
-          tmem_ld32f(lane_base + 128 + 32 * c, dp);
-          tmem_ld_wait();
-          reg_fence_f<32>(x);
-          reg_fence_f<32>(dp);
+          const float* x = xs[cc];
+          const float* dp = dps[cc];
           const uint32_t bits = full ? 0xffffffffu : range_bits(klo_i, khi_i, (long)t * kTile + 32 * c);
           uint32_t pk[16];
 #pragma unroll
@@ -914,7 +971,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bar.comp_ready);
+        mbar_arrive(&bar.comp_ready[half]);
       }
       if (!ok) break;
       if (!wait_all(&bar.acc_done, ucnt & 1)) break;
