@@ -210,7 +210,7 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     attn_bwd_dkdv_kernel<D><<<a.n_units < sms ? a.n_units : sms, kBwdThreads, L::kSmemBytes, st>>>(mq, mk, mv, mdo,
                                                                                                     a);
     if (a.n_slots > 0)
-      attn_bwd_dkdv_reduce_kernel<D><<<dim3(a.nK, a.B * a.Hkv, kTile * D / kReduceElems), 256, 0, st>>>(a);
+      attn_bwd_dkdv_reduce_kernel<D><<<dim3(a.nK, a.B * a.Hkv, kTile * D / 8 / kReduceThreads), kReduceThreads, 0, st>>>(a);
   }
   a.n_units = a.B * a.Hq * a.nQ;
   attn_bwd_dq_kernel<D><<<a.n_units < sms ? a.n_units : sms, kBwdThreads, L::kSmemBytes, st>>>(mq, mk, mv, mdo, a);

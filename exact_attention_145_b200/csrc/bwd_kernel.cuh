@@ -90,7 +90,8 @@ struct BwdArgs {
   // dK/dV plan (workspace, written by the delta kernel's last block):
   const int4* pieces;  // [n_pieces] {key tile, first step, end step, partial slot or -1}
   const int2* tiles;   // [nK] {pieces of the tile, first partial slot or -1}
-  float* part;         // [B * Hkv][n_slots][2][128][D] fp32 partial dV, dK (dK without the scale)
+  float* part;         // [B * Hkv][n_slots][2][D / 4][128] float4: fp32 partial dV, dK (dK without the scale),
+                       // row-interleaved so that a warp's rows are one contiguous 512-byte store
   int n_pieces, n_slots, cap;
   int n_units;
   int* status;
@@ -518,7 +519,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     int ucnt = 0, gstep = 0;
     bool ok = true;
     const float NEG_INF = -__int_as_float(0x7f800000);
-    const float POS_INF = __int_as_float(0x7f800000);
     for (int r = 0; ok && r < rounds; ++r) {
       const int u = unit_of(r);
       if (u < 0) continue;
@@ -552,15 +552,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       auto column_value = [&](int s) -> float {
         const int qt = w.qlo + (w.s0 + s) / a.g, h = w.hk * a.g + (w.s0 + s) % a.g;
         const int typ = row / 64, qi = qt * kTile + 64 * half + row % 64;
-        float val = typ == 0 ? POS_INF : 0.f;
+        // stored negated: -log2e * LSE (-inf for a row with no allowed key
+        // or past Sq, so its weights come out +0) and -delta
+        float val = typ == 0 ? NEG_INF : 0.f;
         if (qi < a.Sq) {
           const int64_t ix = ((int64_t)w.b * a.Hq + h) * a.Sq + qi;
           if (typ == 0) {
             const float l = __ldg(a.lse + ix);
-            // LSE -inf (a row with no allowed key): none of its pairs is allowed either
-            val = l == NEG_INF ? POS_INF : l * kLog2eB;
+            val = l == NEG_INF ? NEG_INF : -l * kLog2eB;
           } else {
-            val = __ldg(a.delta + ix);
+            val = -__ldg(a.delta + ix);
           }
         }
         return val;
@@ -589,25 +590,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           reg_fence_f<32>(x);
           reg_fence_f<32>(dp);
           const uint32_t bits = full ? 0xffffffffu : range_bits(qlo_i, qhi_i, (long)qt * kTile + 32 * c);
-          const float4* l2v = reinterpret_cast<const float4*>(vec + 32 * cc);
-          const float4* dlv = reinterpret_cast<const float4*>(vec + 64 + 32 * cc);
+          const float4* nl2v = reinterpret_cast<const float4*>(vec + 32 * cc);
+          const float4* ndlv = reinterpret_cast<const float4*>(vec + 64 + 32 * cc);
+          const float2 SL2 = make_float2(a.scale_log2, a.scale_log2);
           uint32_t pk[16], dk[16];
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 l4 = l2v[e4], d4 = dlv[e4];
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
-            float pe[4], de[4];
-#pragma unroll
-            for (int z = 0; z < 4; ++z) {
-              const int e = 4 * e4 + z;
-              const float p = ((bits >> e) & 1u) ? bex2(fmaf(x[e], a.scale_log2, -lv[z])) : 0.f;
-              pe[z] = p;
-              de[z] = p * (dp[e] - dv[z]);
+            const float4 l4 = nl2v[e4], d4 = ndlv[e4];
+            const int e = 4 * e4;
+            // P^T = 2^(scale log2e S^T - log2e LSE), dS^T = P^T (dP^T - delta), two columns per op
+            const float2 z0 = fma2(make_float2(x[e], x[e + 1]), SL2, make_float2(l4.x, l4.y));
+            const float2 z1 = fma2(make_float2(x[e + 2], x[e + 3]), SL2, make_float2(l4.z, l4.w));
+            float2 p0 = make_float2(bex2(z0.x), bex2(z0.y)), p1 = make_float2(bex2(z1.x), bex2(z1.y));
+            if (!full) {
+              p0.x = ((bits >> e) & 1u) ? p0.x : 0.f;
+              p0.y = ((bits >> (e + 1)) & 1u) ? p0.y : 0.f;
+              p1.x = ((bits >> (e + 2)) & 1u) ? p1.x : 0.f;
+              p1.y = ((bits >> (e + 3)) & 1u) ? p1.y : 0.f;
             }
-            pk[2 * e4] = pack_bf16x2(pe[0], pe[1]);
-            pk[2 * e4 + 1] = pack_bf16x2(pe[2], pe[3]);
-            dk[2 * e4] = pack_bf16x2(de[0], de[1]);
-            dk[2 * e4 + 1] = pack_bf16x2(de[2], de[3]);
+            const float2 ds0 = mul2(p0, add2(make_float2(dp[e], dp[e + 1]), make_float2(d4.x, d4.y)));
+            const float2 ds1 = mul2(p1, add2(make_float2(dp[e + 2], dp[e + 3]), make_float2(d4.z, d4.w)));
+            pk[2 * e4] = pack_bf16x2(p0.x, p0.y);
+            pk[2 * e4 + 1] = pack_bf16x2(p1.x, p1.y);
+            dk[2 * e4] = pack_bf16x2(ds0.x, ds0.y);
+            dk[2 * e4 + 1] = pack_bf16x2(ds1.x, ds1.y);
           }
           // P^T and dS^T of chunk c -> the first 16 of its own 32 source columns
           tmem_st16(lane_base + 32 * c, *reinterpret_cast<uint32_t(*)[16]>(pk));
@@ -632,8 +638,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (w.slot >= 0) {
           const int grp = w.b * a.Hkv + w.hk;
           float* base = a.part + ((size_t)grp * a.n_slots + w.slot) * 2 * kTile * D;
-          pv = base + (size_t)row * D + c_lo;
-          pkp = base + (size_t)kTile * D + (size_t)row * D + c_lo;
+          pv = base + ((size_t)(c_lo / 4) * kTile + row) * 4;
+          pkp = pv + (size_t)kTile * D;
         }
 #pragma unroll 1
         for (int c = 0; c < D / 2; c += 32) {
@@ -647,8 +653,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // partial of a split key tile: fp32, every row (the reduction skips ragged rows)
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
-              *reinterpret_cast<float4*>(pv + c + e) = make_float4(v0[e], v0[e + 1], v0[e + 2], v0[e + 3]);
-              *reinterpret_cast<float4*>(pkp + c + e) = make_float4(k0[e], k0[e + 1], k0[e + 2], k0[e + 3]);
+              const size_t o4 = (size_t)((c + e) / 4) * kTile * 4;  // next column quad: 128 rows further
+              *reinterpret_cast<float4*>(pv + o4) = make_float4(v0[e], v0[e + 1], v0[e + 2], v0[e + 3]);
+              *reinterpret_cast<float4*>(pkp + o4) = make_float4(k0[e], k0[e + 1], k0[e + 2], k0[e + 3]);
             }
           } else {
 #pragma unroll
@@ -686,34 +693,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // Sums the partials of key tiles that were cut into several pieces, in piece
-// order, and writes dV and scale * dK as bf16. Grid (nK, B * Hkv,
-// 128 * D / 1024): each block sums 1024 consecutive elements (1024 / D rows)
-// of both tiles, one float4 per thread.
-constexpr int kReduceElems = 1024;
+// order, and writes dV and scale * dK as bf16. Grid (nK, B * Hkv, D / 16),
+// 256 threads: thread = (8-column group, row), reading two row-interleaved
+// float4 (coalesced over rows) per tile and writing 16 bytes of bf16.
+constexpr int kReduceThreads = 256;
 template <int D>
-__global__ void __launch_bounds__(256) attn_bwd_dkdv_reduce_kernel(const BwdArgs a) {
+__global__ void __launch_bounds__(kReduceThreads) attn_bwd_dkdv_reduce_kernel(const BwdArgs a) {
   const int t = blockIdx.x, grp = blockIdx.y;
   const int2 tl = a.tiles[t];
   if (tl.x <= 1) return;
   const int b = grp / a.Hkv, hk = grp % a.Hkv;
   const size_t tile_elems = (size_t)kTile * D;
   const float* base = a.part + ((size_t)grp * a.n_slots + tl.y) * 2 * tile_elems;
-  const int idx = blockIdx.z * kReduceElems + threadIdx.x * 4;
-  const int row = idx / D, col = idx % D;
-  float4 sv = make_float4(0.f, 0.f, 0.f, 0.f), sk = sv;
+  const int id = blockIdx.z * kReduceThreads + threadIdx.x;  // < 128 * D / 8
+  const int row = id % kTile, c8 = id / kTile;
+  const size_t o0 = ((size_t)(2 * c8) * kTile + row) * 4, o1 = o0 + (size_t)kTile * 4;
+  float sv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, sk[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   for (int j = 0; j < tl.x; ++j) {
-    const float4 v = *reinterpret_cast<const float4*>(base + (size_t)j * 2 * tile_elems + idx);
-    const float4 k = *reinterpret_cast<const float4*>(base + (size_t)j * 2 * tile_elems + tile_elems + idx);
-    sv.x += v.x; sv.y += v.y; sv.z += v.z; sv.w += v.w;
-    sk.x += k.x; sk.y += k.y; sk.z += k.z; sk.w += k.w;
+    const float* pvj = base + (size_t)j * 2 * tile_elems;
+    const float* pkj = pvj + tile_elems;
+    const float4 v0 = *reinterpret_cast<const float4*>(pvj + o0), v1 = *reinterpret_cast<const float4*>(pvj + o1);
+    const float4 k0 = *reinterpret_cast<const float4*>(pkj + o0), k1 = *reinterpret_cast<const float4*>(pkj + o1);
+    sv[0] += v0.x; sv[1] += v0.y; sv[2] += v0.z; sv[3] += v0.w;
+    sv[4] += v1.x; sv[5] += v1.y; sv[6] += v1.z; sv[7] += v1.w;
+    sk[0] += k0.x; sk[1] += k0.y; sk[2] += k0.z; sk[3] += k0.w;
+    sk[4] += k1.x; sk[5] += k1.y; sk[6] += k1.z; sk[7] += k1.w;
   }
   const long key = (long)t * kTile + row;
   if (key >= a.Skv) return;
+  const int col = 8 * c8;
   __nv_bfloat16* dvr = a.dv + b * a.dv_sb + key * a.dv_ss + (int64_t)hk * a.dv_sh + col;
   __nv_bfloat16* dkr = a.dk + b * a.dk_sb + key * a.dk_ss + (int64_t)hk * a.dk_sh + col;
-  *reinterpret_cast<uint2*>(dvr) = make_uint2(pack_bf16x2(sv.x, sv.y), pack_bf16x2(sv.z, sv.w));
-  *reinterpret_cast<uint2*>(dkr) = make_uint2(pack_bf16x2(sk.x * a.scale, sk.y * a.scale),
-                                              pack_bf16x2(sk.z * a.scale, sk.w * a.scale));
+  uint4 ov, ok;
+  ov.x = pack_bf16x2(sv[0], sv[1]);
+  ov.y = pack_bf16x2(sv[2], sv[3]);
+  ov.z = pack_bf16x2(sv[4], sv[5]);
+  ov.w = pack_bf16x2(sv[6], sv[7]);
+  ok.x = pack_bf16x2(sk[0] * a.scale, sk[1] * a.scale);
+  ok.y = pack_bf16x2(sk[2] * a.scale, sk[3] * a.scale);
+  ok.z = pack_bf16x2(sk[4] * a.scale, sk[5] * a.scale);
+  ok.w = pack_bf16x2(sk[6] * a.scale, sk[7] * a.scale);
+  *reinterpret_cast<uint4*>(dvr) = ov;
+  *reinterpret_cast<uint4*>(dkr) = ok;
 }
 
 // ---------------------------------------------------------------- dQ
@@ -921,8 +942,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       const int64_t rix = ((int64_t)w.b * a.Hq + w.h) * a.Sq + min(qi, a.Sq - 1);
       const float lse = a.lse[rix];
-      const float l2 = (!valid || lse == NEG_INF) ? __int_as_float(0x7f800000) : lse * kLog2eB;
-      const float dlt = a.delta[rix];
+      // negated row values: -log2e * LSE (-inf: no allowed key / past Sq, weights +0) and -delta
+      const float nl2 = (!valid || lse == NEG_INF) ? NEG_INF : -lse * kLog2eB;
+      const float ndl = -a.delta[rix];
       // keys this query sees: [q_pos - wl, q_pos + wr]
       const long q_pos = (long)qi + a.q_offset;
       long klo_i = 0, khi_i = (long)a.Skv - 1;
@@ -954,17 +976,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const float* x = xs[cc];
           const float* dp = dps[cc];
           const uint32_t bits = full ? 0xffffffffu : range_bits(klo_i, khi_i, (long)t * kTile + 32 * c);
+          const float2 SL2 = make_float2(a.scale_log2, a.scale_log2), NL2 = make_float2(nl2, nl2);
+          const float2 NDL = make_float2(ndl, ndl);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            float de[2];
-#pragma unroll
-            for (int z = 0; z < 2; ++z) {
-              const bool on = (bits >> (e + z)) & 1u;
-              const float p = on ? bex2(fmaf(x[e + z], a.scale_log2, -l2)) : 0.f;
-              de[z] = p * (dp[e + z] - dlt);
+            // dS = 2^(scale log2e S - log2e LSE) (dP - delta), two columns per op
+            const float2 z = fma2(make_float2(x[e], x[e + 1]), SL2, NL2);
+            float2 p = make_float2(bex2(z.x), bex2(z.y));
+            if (!full) {
+              p.x = ((bits >> e) & 1u) ? p.x : 0.f;
+              p.y = ((bits >> (e + 1)) & 1u) ? p.y : 0.f;
             }
-            pk[e / 2] = pack_bf16x2(de[0], de[1]);
+            const float2 ds = mul2(p, add2(make_float2(dp[e], dp[e + 1]), NDL));
+            pk[e / 2] = pack_bf16x2(ds.x, ds.y);
           }
           // dS of chunk c -> the first 16 of its own 32 source columns
           tmem_st16(lane_base + 32 * c, *reinterpret_cast<uint32_t(*)[16]>(pk));
