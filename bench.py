@@ -590,7 +590,7 @@ def main():
     ap.add_argument("--workload", default=PRIMARY, choices=[k for k, v in W.WORKLOADS.items()
                                                           if isinstance(v, W.Prefill)])
     ap.add_argument("--secondary-steps", type=int, default=200)
-    ap.add_argument("--profile", default=None, choices=list(W.WORKLOADS) + ["block_mask", "backward_" + PRIMARY],
+    ap.add_argument("--profile", default=None, choices=list(W.WORKLOADS) + ["block_mask", "backward_" + PRIMARY, "with_kvcache"],
                     help="run --steps eager steps of one workload (for ncu captures); prints no JSON line")
     ap.add_argument("--plumbing-check", action="store_true",
                     help="CPU only: rehearse the N-rank launch, barrier and max over ranks over gloo")
@@ -753,6 +753,8 @@ def profile_arm(args):
         d = W.make_prefill_inputs(w)
         doc = torch.from_numpy(d["doc_id"]).to(device)
         step = lambda i: ea.attn_build_block_mask(w.S, w.S, doc_id=doc)  # noqa: E731
+    elif name == "with_kvcache":
+        step = kvcache_setup(torch, ea, device, 0)["step"]
     elif name.startswith("backward_"):
         step = backward_setup(torch, ea, W.WORKLOADS[name[len("backward_"):]], device, 0)["step"]
     elif isinstance(W.WORKLOADS[name], W.Decode):

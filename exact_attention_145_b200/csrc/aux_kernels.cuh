@@ -25,6 +25,7 @@ struct MaskArgs {
 // Only in-range positions of ragged edge tiles count.
 constexpr int kMaskThreads = 128;
 constexpr int kKvPerCta = 8;
+constexpr int kRunPerThread = 8;  // ids per thread per shared-memory segment of doc_runs_kernel
 
 // Window forms (none, causal, window): one thread per tile, exact interval
 // arithmetic. The keys a query at position p may see form the window
@@ -86,6 +87,13 @@ __global__ void __launch_bounds__(kMaskThreads) classify_doc_kernel(MaskArgs a) 
   const int rows = min(a.blk_q, a.Sq - q0);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int k_first = kt0 * a.blk_kv, k_end = min(kt1 * a.blk_kv, a.Skv);
+  if (k_first > q0 + rows - 1) {
+    // every key of these tiles lies past the last query of the row tile:
+    // all empty under the causal document mask, no ids needed
+    // (head slice 0, like the classification below; the compaction copies it)
+    for (int kt = kt0 + threadIdx.x; kt < kt1; kt += blockDim.x) a.cls[(int64_t)qt * a.nK + kt] = 0;
+    return;
+  }
   for (int c = threadIdx.x; c < k_end - k_first; c += blockDim.x) doc_k[c] = a.doc_id[k_first + c];
   // id range of the query tile
   int lo = 0x7fffffff, hi = -0x7fffffff - 1;
@@ -222,46 +230,74 @@ __global__ void __launch_bounds__(kOrderThreads) row_order_kernel(const MaskArgs
 // last run starts are combined with a block-wide max scan.
 constexpr int kRunThreads = 1024;
 __global__ void __launch_bounds__(kRunThreads) doc_runs_kernel(const MaskArgs a) {
+  // The ids are staged segment by segment in shared memory with coalesced
+  // loads (each thread then scans kRunPerThread consecutive ids there), and
+  // the run starts go back through the same buffer with coalesced stores.
+  __shared__ int seg[kRunThreads * kRunPerThread];
   __shared__ int warp_max[kRunThreads / 32];
   const int b = blockIdx.x;
   const int32_t* doc = a.doc_id + (int64_t)b * a.doc_bstride;
   int32_t* out = a.doc_start + (int64_t)b * a.Sq;
   const int S = a.Sq;
-  const int chunk = (S + kRunThreads - 1) / kRunThreads;
-  const int i0 = min(S, (int)threadIdx.x * chunk), i1 = min(S, i0 + chunk);
-  int last = -1;
-  bool decreasing = false;
-  for (int i = i0; i < i1; ++i) {
-    const int d = doc[i];
-    if (i == 0 || d != doc[i - 1]) last = i;
-    if (i > 0 && d < doc[i - 1]) decreasing = true;
-  }
-  // inclusive max scan of `last` over threads: warps, then the warp totals
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
-  int incl = last;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl = max(incl, v);
-  }
-  if (lane == 31) warp_max[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = warp_max[lane];
+  constexpr int kSeg = kRunThreads * kRunPerThread;
+  int carry = -1;        // last run start before the segment
+  int prev_id = 0;       // id just before the segment (valid when seg0 > 0)
+  bool decreasing = false;
+  for (int seg0 = 0; seg0 < S; seg0 += kSeg) {
+    const int n = min(kSeg, S - seg0);
+    for (int c = threadIdx.x; c < n; c += kRunThreads) seg[c] = doc[seg0 + c];
+    __syncthreads();
+    const int i0 = min(n, (int)threadIdx.x * kRunPerThread), i1 = min(n, i0 + kRunPerThread);
+    // ids read before any thread rewrites the buffer: the one before this
+    // thread's range, and the segment's last
+    const int first_prev = i0 > 0 ? seg[i0 - 1] : prev_id;
+    const int last_id = seg[n - 1];
+    int last = -1;
+    for (int i = i0; i < i1; ++i) {
+      const int d = seg[i];
+      const int dp = i > 0 ? seg[i - 1] : prev_id;
+      const bool start = (seg0 + i == 0) || d != dp;
+      if (start) last = seg0 + i;
+      if (seg0 + i > 0 && d < dp) decreasing = true;
+    }
+    // inclusive max scan of `last` over threads: warps, then the warp totals
+    int incl = last;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, w, off);
-      if (lane >= off) w = max(w, v);
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl = max(incl, v);
     }
-    warp_max[lane] = w;  // inclusive over warps 0..lane
-  }
-  __syncthreads();
-  const int before_warp = warp > 0 ? warp_max[warp - 1] : -1;
-  const int excl_lane = __shfl_up_sync(0xffffffffu, incl, 1);
-  int cur = max(before_warp, lane > 0 ? excl_lane : -1);  // last run start before this chunk
-  for (int i = i0; i < i1; ++i) {
-    if (i == 0 || doc[i] != doc[i - 1]) cur = i;
-    out[i] = cur;
+    if (lane == 31) warp_max[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_max[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, w, off);
+        if (lane >= off) w = max(w, v);
+      }
+      warp_max[lane] = w;  // inclusive over warps 0..lane
+    }
+    __syncthreads();
+    const int before_warp = warp > 0 ? warp_max[warp - 1] : -1;
+    const int excl_lane = __shfl_up_sync(0xffffffffu, incl, 1);
+    int cur = max(carry, max(before_warp, lane > 0 ? excl_lane : -1));
+    const int seg_last = warp_max[kRunThreads / 32 - 1];
+    // run starts in place of the ids (each thread reads and rewrites only its
+    // own range; the id before it was saved above)
+    int dp = first_prev;
+    for (int i = i0; i < i1; ++i) {
+      const int d = seg[i];
+      if ((seg0 + i == 0) || d != dp) cur = seg0 + i;
+      dp = d;
+      seg[i] = cur;
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < n; c += kRunThreads) out[seg0 + c] = seg[c];
+    carry = max(carry, seg_last);
+    prev_id = last_id;
+    __syncthreads();
   }
   const int any_dec = __syncthreads_or(decreasing ? 1 : 0);
   if (threadIdx.x == 0) a.doc_sorted[b] = any_dec ? 0 : 1;
