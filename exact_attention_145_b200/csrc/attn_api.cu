@@ -599,9 +599,10 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
   }
   if (p->block_mask) {
     const attn_block_mask* bm = p->block_mask;
-    if (bm->blk_q != kRows || bm->blk_kv != kKeys || bm->Sq != p->Sq || bm->Skv != p->Skv || !bm->cls ||
-        bm->n_q_tiles != nQ || bm->n_kv_tiles != nK || !bm->part_cnt || !bm->part_idx || !bm->full_cnt ||
-        !bm->full_idx)
+    // 128 x 128 tables, or 256 x 128: one table row per two-subtile CTA
+    if ((bm->blk_q != kRows && bm->blk_q != 2 * kRows) || bm->blk_kv != kKeys || bm->Sq != p->Sq ||
+        bm->Skv != p->Skv || !bm->cls || bm->n_q_tiles != (p->Sq + bm->blk_q - 1) / bm->blk_q ||
+        bm->n_kv_tiles != nK || !bm->part_cnt || !bm->part_idx || !bm->full_cnt || !bm->full_idx)
       return ATTN_ERR_INVALID_ARG;
     if ((bm->Bm != 1 && bm->Bm != p->B) || (bm->Hm != 1 && bm->Hm != p->Hq)) return ATTN_ERR_INVALID_ARG;
     if (p->mask.kind == ATTN_MASK_DOCUMENT && (!bm->doc_start || !bm->doc_sorted)) return ATTN_ERR_INVALID_ARG;
@@ -643,6 +644,8 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
   if (p->block_mask) {
     a.bm_Bm = p->block_mask->Bm;
     a.bm_Hm = p->block_mask->Hm;
+    a.bm_rows = p->block_mask->blk_q;
+    a.bm_nQ = p->block_mask->n_q_tiles;
     a.bm_row_order = p->block_mask->row_order;
     a.bm_doc_start = p->block_mask->doc_start;
     a.bm_doc_sorted = p->block_mask->doc_sorted;
@@ -665,6 +668,9 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
   a.status = p->status;
   a.pair_heads = (a.g % 2 == 0) ? 1 : 0;
   a.n_row_units = a.pair_heads ? nQ : (nQ + 1) / 2;
+  // a 256-row table in the paired-head layout: each table row is two units
+  // (the second of an odd last row is empty)
+  if (p->block_mask && a.pair_heads && a.bm_rows == 2 * kRows) a.n_row_units = 2 * a.bm_nQ;
 
   CUtensorMap mq, mk, mv, mo;
   const uint64_t dq[4] = {(uint64_t)p->D, (uint64_t)p->Sq, (uint64_t)p->Hq, (uint64_t)p->B};

@@ -84,6 +84,7 @@ struct FwdArgs {
   const uint8_t* bm_cls;  // [Bm][Hm][nQ][nK] class tables or nullptr
   const int32_t *bm_part_cnt, *bm_part_idx, *bm_full_cnt, *bm_full_idx;  // ascending kv-tile lists
   int bm_Bm, bm_Hm;       // slices of the block mask (1 = shared by every batch / head)
+  int bm_rows, bm_nQ;     // query rows per table row (128 or 256) and table rows
   const int32_t* bm_row_order;   // [Bm][nQ] q-tiles heaviest first, or nullptr
   const int32_t* bm_doc_start;   // [Bm][Sq] document run starts (document masks)
   const int32_t* bm_doc_sorted;  // [Bm] 1: every document is one run of ids
@@ -230,10 +231,13 @@ __device__ __forceinline__ Work map_work(const FwdArgs& a, int u) {
     const int hu = rem % HU;
     int rt = a.n_row_units - 1 - qi;
     if (a.bm_row_order != nullptr && a.pair_heads) {
-      // a caller-written order entry outside the q-tiles falls back to the
-      // default order (the producer reports it as a bad mask)
-      const int o = __ldg(a.bm_row_order + (int64_t)(a.bm_Bm == 1 ? 0 : w.b) * a.nQ + qi);
-      if (o >= 0 && o < a.n_row_units) rt = o;
+      // Table rows in the table's order; a 256-row table row expands into
+      // its two 128-row tiles (units past the last tile are empty). A
+      // caller-written order entry outside the table falls back to the
+      // default order (the producer reports it as a bad mask).
+      const int sub = a.bm_rows / kRows;
+      const int o = __ldg(a.bm_row_order + (int64_t)(a.bm_Bm == 1 ? 0 : w.b) * a.bm_nQ + qi / sub);
+      if (o >= 0 && o < a.bm_nQ) rt = o * sub + qi % sub;
     }
     if (a.pair_heads) {
       w.head0 = 2 * hu;
@@ -274,7 +278,7 @@ __device__ __forceinline__ int tile_class(const FwdArgs& a, const Work& w, int s
     const bool ragged = c0 + kKeys > a.Skv;
     int cls;
     if constexpr (BM) {
-      cls = a.bm_cls[(bm_slice(a, w.b, w_head(w, s)) * a.nQ + r0 / kRows) * a.nK + t];
+      cls = a.bm_cls[(bm_slice(a, w.b, w_head(w, s)) * a.bm_nQ + r0 / a.bm_rows) * a.nK + t];
     } else if (a.mask == MASK_NONE) {
       cls = 2;
     } else {
@@ -363,8 +367,8 @@ __device__ __forceinline__ int walker_init(const FwdArgs& a, const Work& w, Tile
   } else {
     // row q-tile of each subtile within its (batch, head) slice; the second
     // list is needed only when the subtiles differ in rows or in slice
-    const int64_t q0 = bm_slice(a, w.b, w.head0) * a.nQ + w.row00 / kRows;
-    const int64_t q1 = bm_slice(a, w.b, w.head1) * a.nQ + w.row01 / kRows;
+    const int64_t q0 = bm_slice(a, w.b, w.head0) * a.bm_nQ + w.row00 / a.bm_rows;
+    const int64_t q1 = bm_slice(a, w.b, w.head1) * a.bm_nQ + w.row01 / a.bm_rows;
     // counts are clamped to a row's length, so lists are never read past it
     if (w.row00 < a.Sq) {
       tw.np0 = min(max(__ldg(a.bm_part_cnt + q0), 0), a.nK);
@@ -1365,12 +1369,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qi = u / (a.B * (a.pair_heads ? a.Hq / 2 : a.Hq));
         bool bad = false;
         if (a.bm_row_order != nullptr && a.pair_heads) {
-          const int o = __ldg(a.bm_row_order + (int64_t)(a.bm_Bm == 1 ? 0 : w.b) * a.nQ + qi);
-          bad = o < 0 || o >= a.n_row_units;
+          const int o = __ldg(a.bm_row_order + (int64_t)(a.bm_Bm == 1 ? 0 : w.b) * a.bm_nQ + qi / (a.bm_rows / kRows));
+          bad = o < 0 || o >= a.bm_nQ;
         }
         for (int s = 0; s < 2; ++s) {
           if (w_row0(w, s) >= a.Sq) continue;
-          const int64_t q = bm_slice(a, w.b, w_head(w, s)) * a.nQ + w_row0(w, s) / kRows;
+          const int64_t q = bm_slice(a, w.b, w_head(w, s)) * a.bm_nQ + w_row0(w, s) / a.bm_rows;
           const int pc = __ldg(a.bm_part_cnt + q), fc = __ldg(a.bm_full_cnt + q);
           bad |= pc < 0 || pc > a.nK || fc < 0 || fc > a.nK;
         }

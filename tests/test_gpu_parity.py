@@ -541,3 +541,36 @@ def test_full_mqa_paged_decode_sampled_sequences():
                cache_seqlens=d["cache_seqlens"][pick])
     o_ref, lse_ref = oracle.decode(sub["q"], sub["k_cache"], sub["v_cache"], sub["block_table"], sub["cache_seqlens"])
     compare(o[pick], o_ref, lse[pick], lse_ref, "full decode")
+
+
+# ------------------------------------------------------------ 256 x 128 tables
+
+@pytest.mark.parametrize("S,Hq,Hkv,docs", [(300, 4, 2, None), (1000, 8, 2, [300, 77, 500, 123]),
+                                            (900, 3, 1, [450, 450]), (700, 2, 2, None)])
+def test_block_mask_256_row_tables(S, Hq, Hkv, docs):
+    """A 256 x 128 table (one row per two-subtile CTA, the talk's Blackwell
+    block-sparse granularity) gives the same result as the 128 x 128 table
+    and the oracle; odd tile counts leave an empty unit, odd groups use the
+    256-row single-head units."""
+    q, k, v = (W.normal_bf16(500 + S, (1, S, Hq, 128)), W.normal_bf16(501 + S, (1, S, Hkv, 128)),
+               W.normal_bf16(502 + S, (1, S, Hkv, 128)))
+    kw, okw = {}, {}
+    if docs is None:
+        kw["causal"] = True
+        okw = dict(mask=oracle.MASK_CAUSAL, window=(-1, 0))
+        bm256 = ea.attn_build_block_mask(S, S, causal=True, blk_q=256, blk_kv=128, device=torch.device("cuda"))
+        bm128 = ea.attn_build_block_mask(S, S, causal=True, device=torch.device("cuda"))
+    else:
+        doc = W.doc_ids_from_lengths(docs)
+        kw["doc_id"] = torch.from_numpy(doc).cuda()
+        okw = dict(mask=oracle.MASK_DOCUMENT, doc_id=doc)
+        bm256 = ea.attn_build_block_mask(S, S, doc_id=kw["doc_id"], blk_q=256, blk_kv=128)
+        bm128 = ea.attn_build_block_mask(S, S, doc_id=kw["doc_id"])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o1, l1 = ea.attn_fwd(dev_bf16(q), dev_bf16(k), dev_bf16(v), block_mask=bm256, status=status, **kw)
+    o2, l2 = ea.attn_fwd(dev_bf16(q), dev_bf16(k), dev_bf16(v), block_mask=bm128, **kw)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    ro, rl = oracle.attn(q, k, v, **okw)
+    compare(host_f64(o1)[0], ro[0], l1.cpu().numpy().astype(np.float64)[0], rl[0], "256-row table S=%d" % S)
