@@ -718,8 +718,8 @@ def secondary(torch, ea, device, stream, peaks, rank, barrier, max_over_ranks, w
         "flops_rule": "10*D*pairs (S, dP, dV, dK, dQ products)",
         "roofline": {"bound": "tensor", "achieved": ach, "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
                      "frac": ach / float(peaks["bf16_tflops"]), "traffic": None},
-        "kernels": "delta_kernel, attn_bwd_dkdv_kernel<128>, attn_bwd_dq_kernel<128>"}
-    launches += 3 * bsteps
+        "kernels": "delta_kernel, attn_bwd_dkdv_kernel<128>, attn_bwd_dkdv_reduce_kernel<128>, attn_bwd_dq_kernel<128>"}
+    launches += 4 * bsteps  # delta (+ plan), dK/dV, dK/dV reduce (split tiles), dQ
     w = W.WORKLOADS["mqa_paged_decode_b32_kv32768"]
     s = decode_setup(torch, ea, w, device, seed_shift=rank_seed_shift(rank))
     t, _ = graph_time(torch, s["step"], steps, stream, 5, barrier)

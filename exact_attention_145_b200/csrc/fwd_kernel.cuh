@@ -172,6 +172,7 @@ struct Barriers {
 enum : int {
   kTraceRoles = 11, TR_TMA = 9,
   EV_S_WAIT = 1, EV_S_READY = 2, EV_P_DONE = 3, EV_O_WAIT = 4, EV_EPI_BEGIN = 5, EV_EPI_END = 6,
+  EV_HALF_A_DONE = 7, EV_SB_WAIT = 8, EV_SB_READY = 9,
   EV_Q_FULL = 10, EV_PV = 11, EV_QK = 12, EV_P_WAIT = 13, EV_MMA_END = 14, EV_PV_ISSUED = 15,
   EV_Q_LOAD = 20, EV_KV_LOAD = 21, EV_KERNEL_END = 30
 };
@@ -1045,8 +1046,10 @@ __device__ __forceinline__ bool softmax_step_halves(const FwdArgs& a, const Work
 #pragma unroll 1
   for (int h = 0; h < 2; ++h) {
     if (h == 1 && !b_ready) {
+      ATTN_TRACE_REC(threadIdx.x / 32, EV_SB_WAIT, g);
       if (!__all_sync(0xffffffffu, mbar_wait_spin(&bar.s_b_ready[s], par, abort_flag))) return false;
       tc_fence_after();
+      ATTN_TRACE_REC(threadIdx.x / 32, EV_SB_READY, g);
     }
     float x[64];
     float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
@@ -1131,6 +1134,7 @@ __device__ __forceinline__ bool softmax_step_halves(const FwdArgs& a, const Work
     tmem_st_wait();
     tc_fence_before();
     mbar_arrive(h == 0 ? &bar.p_ready[s] : &bar.p_b_ready[s]);
+    if (h == 0) ATTN_TRACE_REC(threadIdx.x / 32, EV_HALF_A_DONE, g);
     acc0 = add2(acc0, acc1);
     st.l = st.l * alpha + (acc0.x + acc0.y);
   }
