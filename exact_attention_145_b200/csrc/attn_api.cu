@@ -658,6 +658,7 @@ attn_status attn_fwd(const attn_fwd_params* p, void* stream) {
   a.nK = nK;
   a.mod = p->mod;
   a.softcap = p->softcap;
+  a.softcap_k1 = p->softcap > 0.f ? a.scale / p->softcap : 0.f;
   a.alibi = p->alibi_slopes;
   a.alibi_bstride = p->alibi_batch_stride;
   a.o = static_cast<__nv_bfloat16*>(p->o);
@@ -783,6 +784,7 @@ attn_status attn_decode(const attn_decode_params* p, void* workspace, size_t wor
   a.wl = a.wr = -1;
   a.mod = p->mod;
   a.softcap = p->softcap;
+  a.softcap_k1 = p->softcap > 0.f ? a.scale / p->softcap : 0.f;
   a.alibi = p->alibi_slopes;
   a.alibi_bstride = p->alibi_batch_stride;
   a.status = p->status;

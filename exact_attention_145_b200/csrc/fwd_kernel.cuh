@@ -91,6 +91,7 @@ struct FwdArgs {
   int nQ, nK;
   int mod;
   float softcap;
+  float softcap_k1;  // scale / softcap (the tanh argument per raw score)
   const float* alibi;
   int alibi_bstride;
   // prefill outputs
@@ -312,19 +313,42 @@ struct TileWalker {
   int np0, nf0, np1, nf1, ip0, if0, ip1, if1;
 };
 
-__device__ __forceinline__ int list_head(const int32_t* l, int n, int i) { return i < n ? __ldg(l + i) : 0x7fffffff; }
+// Walk order over the key tiles of a unit. Ascending by default; descending
+// (from the diagonal back) for prefill with ALiBi, whose bias grows towards
+// the query: walked upwards, a row's max would rise by up to slope x 128 per
+// tile (log2 units), far past the rescale threshold, and every tile would
+// redo its exponentials and rescale O. Walked downwards, the first tiles
+// hold the largest biases and later ones rarely exceed them.
+template <bool DECODE, int MOD>
+constexpr bool kDescWalk = !DECODE && MOD == MOD_ALIBI;
+constexpr int kWalkEnd = 0x7fffffff;  // walker_peek past the last tile
 
+// Head i of an ascending list of n entries, taken from the front or the back.
+template <bool DESC>
+__device__ __forceinline__ int list_head(const int32_t* l, int n, int i) {
+  if (i >= n) return DESC ? -1 : kWalkEnd;
+  return __ldg(l + (DESC ? n - 1 - i : i));
+}
+
+template <bool DESC>
 __device__ __forceinline__ int walker_peek(const TileWalker& tw) {
-  return min(min(list_head(tw.p0, tw.np0, tw.ip0), list_head(tw.f0, tw.nf0, tw.if0)),
-             min(list_head(tw.p1, tw.np1, tw.ip1), list_head(tw.f1, tw.nf1, tw.if1)));
+  const int a0 = list_head<DESC>(tw.p0, tw.np0, tw.ip0), b0 = list_head<DESC>(tw.f0, tw.nf0, tw.if0);
+  const int a1 = list_head<DESC>(tw.p1, tw.np1, tw.ip1), b1 = list_head<DESC>(tw.f1, tw.nf1, tw.if1);
+  if constexpr (DESC) {
+    const int m = max(max(a0, b0), max(a1, b1));
+    return m < 0 ? kWalkEnd : m;
+  } else {
+    return min(min(a0, b0), min(a1, b1));
+  }
 }
 
 // Consumes tile t from every list whose head it is.
+template <bool DESC>
 __device__ __forceinline__ void walker_pop(TileWalker& tw, int t) {
-  if (list_head(tw.p0, tw.np0, tw.ip0) == t) ++tw.ip0;
-  if (list_head(tw.f0, tw.nf0, tw.if0) == t) ++tw.if0;
-  if (list_head(tw.p1, tw.np1, tw.ip1) == t) ++tw.ip1;
-  if (list_head(tw.f1, tw.nf1, tw.if1) == t) ++tw.if1;
+  if (list_head<DESC>(tw.p0, tw.np0, tw.ip0) == t) ++tw.ip0;
+  if (list_head<DESC>(tw.f0, tw.nf0, tw.if0) == t) ++tw.if0;
+  if (list_head<DESC>(tw.p1, tw.np1, tw.ip1) == t) ++tw.ip1;
+  if (list_head<DESC>(tw.f1, tw.nf1, tw.if1) == t) ++tw.if1;
 }
 
 // Tile range [lo, hi] of the window form q_pos - left <= kv <= q_pos + right
@@ -345,8 +369,8 @@ __device__ __forceinline__ bool subtile_range(const FwdArgs& a, const Work& w, i
 }
 
 // Sets up the walk of one unit; returns the number of steps and leaves
-// tw.t on the first tile.
-template <bool DECODE, bool BM>
+// tw.t on the first tile (the lowest, or the highest with DESC).
+template <bool DECODE, bool BM, bool DESC = false>
 __device__ __forceinline__ int walker_init(const FwdArgs& a, const Work& w, TileWalker& tw) {
   tw.np0 = tw.nf0 = tw.np1 = tw.nf1 = tw.ip0 = tw.if0 = tw.ip1 = tw.if1 = 0;
   tw.p0 = tw.f0 = tw.p1 = tw.f1 = nullptr;
@@ -363,7 +387,7 @@ __device__ __forceinline__ int walker_init(const FwdArgs& a, const Work& w, Tile
     // the two subtile ranges overlap or touch (rows differ by at most one tile)
     const int lo = e0 ? (e1 ? min(lo0, lo1) : lo0) : lo1;
     const int hi = e0 ? (e1 ? max(hi0, hi1) : hi0) : hi1;
-    tw.t = lo;
+    tw.t = DESC ? hi : lo;
     return hi - lo + 1;
   } else {
     // row q-tile of each subtile within its (batch, head) slice; the second
@@ -386,23 +410,23 @@ __device__ __forceinline__ int walker_init(const FwdArgs& a, const Work& w, Tile
     // count the union, then rewind
     int n = 0;
     TileWalker c = tw;
-    for (int t = walker_peek(c); t != 0x7fffffff; t = walker_peek(c)) {
-      walker_pop(c, t);
+    for (int t = walker_peek<DESC>(c); t != kWalkEnd; t = walker_peek<DESC>(c)) {
+      walker_pop<DESC>(c, t);
       ++n;
     }
-    tw.t = walker_peek(tw);
+    tw.t = walker_peek<DESC>(tw);
     return n;
   }
 }
 
 // Advances a prefill walk to the next tile.
-template <bool BM>
+template <bool BM, bool DESC = false>
 __device__ __forceinline__ void walker_next(TileWalker& tw) {
   if constexpr (!BM) {
-    ++tw.t;
+    tw.t += DESC ? -1 : 1;
   } else {
-    walker_pop(tw, tw.t);
-    tw.t = walker_peek(tw);
+    walker_pop<DESC>(tw, tw.t);
+    tw.t = walker_peek<DESC>(tw);
   }
 }
 
@@ -505,9 +529,10 @@ constexpr float kTanhA7 = -17.0f / 315.0f;
 // scores into log2-domain scores:
 //   softcap: x = c*log2(e) * tanh(s*scale/c);  alibi: x = s*scale*log2(e) + slope*log2(e)*(kv - q_pos)
 template <bool DECODE, int MOD>
-__device__ __forceinline__ void mod_chunk(const FwdArgs& a, const Work& w, int s, int row, int t, int c, float* x) {
+__device__ __forceinline__ void mod_chunk(const FwdArgs& a, const Work& w, int s, int row, int t, int c, float* x,
+                                          float off = 0.0f) {
   if constexpr (MOD == MOD_SOFTCAP) {
-    const float k1 = a.scale / a.softcap;
+    const float k1 = a.softcap_k1;
     const float cl = a.softcap * kLog2e;
     float smax = 0.f;
 #pragma unroll
@@ -553,7 +578,8 @@ __device__ __forceinline__ void mod_chunk(const FwdArgs& a, const Work& w, int s
                               : (long)(w_row0(w, s) + row) + a.q_offset;
     const int head = w_head(w, s) + (DECODE ? row % a.g : 0);
     const float slope = a.alibi[(int64_t)w.b * a.alibi_bstride + min(head, a.Hq - 1)] * kLog2e;
-    const float base = slope * (float)((long)t * kKeys + 32 * c - q_pos);
+    // off (0, or minus the row's reference max) rides along with the bias
+    const float base = slope * (float)((long)t * kKeys + 32 * c - q_pos) + off;
     const float2 SC = make_float2(a.scale_log2, a.scale_log2), SL = make_float2(slope, slope);
     const float2 B = make_float2(base, base);
 #pragma unroll
@@ -678,11 +704,14 @@ __device__ __forceinline__ bool mask_chunk(const FwdArgs& a, const MaskRow& m, i
 
 // Exponentials of one 32-column chunk (16 pairs) against reference max -nmu,
 // packed to bf16 pairs; sums and the chunk max are accumulated on the way.
+// AFFINE false: x already holds the exponents (MULT and NMU unused).
+template <bool AFFINE = true>
 __device__ __forceinline__ void exp_chunk(const float* x, float2 MULT, float2 NMU, uint32_t* pk, float2& acc0,
                                           float2& acc1) {
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    const float2 arg = fma2(make_float2(x[2 * j], x[2 * j + 1]), MULT, NMU);
+    const float2 arg = AFFINE ? fma2(make_float2(x[2 * j], x[2 * j + 1]), MULT, NMU)
+                              : make_float2(x[2 * j], x[2 * j + 1]);
     float2 e;
     if (exp_on_fma(j)) {
       e = exp2_poly2(arg);
@@ -934,6 +963,9 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
 // whole-tile schedule is faster (the half schedule measured 5 % slower).
 template <bool DECODE, int MOD>
 constexpr bool kHalfTiles = !DECODE && MOD != MOD_NONE && MOD != MOD_RELU;
+// Half-tile softmax: fold minus the reference max into the ALiBi bias.
+template <int MOD>
+constexpr bool kFoldRef = MOD == MOD_ALIBI;
 
 // With half tiles: P for keys
 // 0-63 goes to S(s) columns [0, 32) and P for keys 64-127 to [64, 96), so:
@@ -992,7 +1024,7 @@ __device__ __forceinline__ float stream_half(const FwdArgs& a, const Work& w, in
 // exponentials once the reference is known.
 template <int MOD, bool MASKED, bool BM>
 __device__ __forceinline__ float prepare_half(const FwdArgs& a, const Work& w, int s, int row, int t, uint32_t tS,
-                                              int h, float* x) {
+                                              int h, float* x, float off) {
   const float NEG_INF = -__int_as_float(0x7f800000);
   MaskRow mr;
   if constexpr (MASKED) mr = mask_row<false, BM>(a, w, s, row, t);
@@ -1005,7 +1037,7 @@ __device__ __forceinline__ float prepare_half(const FwdArgs& a, const Work& w, i
 #pragma unroll
   for (int cc = 0; cc < 2; ++cc) {
     const int c = 2 * h + cc;
-    if constexpr (MOD != MOD_NONE) mod_chunk<false, MOD>(a, w, s, row, t, c, x + 32 * cc);
+    if constexpr (MOD != MOD_NONE) mod_chunk<false, MOD>(a, w, s, row, t, c, x + 32 * cc, off);
     if constexpr (MASKED) (void)mask_chunk<false, BM>(a, mr, t, c, x + 32 * cc);
     mc = fmaxf(mc, chunk_max(x + 32 * cc));
   }
@@ -1061,6 +1093,7 @@ __device__ __forceinline__ bool softmax_step_halves(const FwdArgs& a, const Work
     float x[64];
     float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
     float mh;
+    float xref = 0.0f;  // the scores in x are relative to this (ALiBi with a reference max)
     const bool have_ref = __all_sync(0xffffffffu, st.m != NEG_INF);
     bool guessed = false;
     if (cls == 0) {
@@ -1087,18 +1120,26 @@ __device__ __forceinline__ bool softmax_step_halves(const FwdArgs& a, const Work
       }
       guessed = true;
     } else {
+      // ALiBi with a reference max: minus the reference joins the bias, so
+      // the half's scores come out as exponents (one packed op per pair
+      // fewer); xref is what they are relative to.
+      const float off = (kFoldRef<MOD> && have_ref) ? -st.m : 0.0f;
+      xref = -off;
       float mc;
       if (cls == 2)
-        mc = prepare_half<MOD, false, BM>(a, w, s, row, t, tS, h, x);
+        mc = prepare_half<MOD, false, BM>(a, w, s, row, t, tS, h, x, off);
       else
-        mc = prepare_half<MOD, true, BM>(a, w, s, row, t, tS, h, x);
-      mh = mc * mult;
+        mc = prepare_half<MOD, true, BM>(a, w, s, row, t, tS, h, x, off);
+      mh = mc * mult + xref;
       if (have_ref) {
         const float2 NMU = make_float2(-st.m, -st.m);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
-          exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
+          if constexpr (kFoldRef<MOD>)
+            exp_chunk<false>(x + 32 * c, MULT, NMU, pk, acc0, acc1);
+          else
+            exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
           tmem_st16(tS + 64 * h + 16 * c, pk);
         }
       }
@@ -1109,7 +1150,7 @@ __device__ __forceinline__ bool softmax_step_halves(const FwdArgs& a, const Work
       const float m_new = fmaxf(st.m, mh);
       alpha = (m_new == NEG_INF || st.m == NEG_INF) ? (st.m == NEG_INF ? 0.0f : 1.0f) : ex2(st.m - m_new);
       st.m = m_new;
-      const float nmu = (m_new == NEG_INF) ? 0.0f : -m_new;
+      const float nmu = (m_new == NEG_INF) ? 0.0f : xref - m_new;
       const float2 NMU = make_float2(nmu, nmu);
       acc0 = acc1 = make_float2(0.f, 0.f);
       tmem_st_wait();  // the optimistic P stores land before they are overwritten
@@ -1393,7 +1434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       TileWalker tw;
-      const int n = walker_init<DECODE, BM>(a, w, tw);
+      const int n = walker_init<DECODE, BM, kDescWalk<DECODE, MOD>>(a, w, tw);
       if (n == 0) continue;
       if (qcnt > 0 && !wait_all(&bar.q_empty, (qcnt - 1) & 1)) {
         ok = false;
@@ -1462,7 +1503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (DECODE)
           ++tw.t;
         else
-          walker_next<BM>(tw);
+          walker_next<BM, kDescWalk<DECODE, MOD>>(tw);
       }
     }
     // Drain: on an abort, wait (bounded) for every copy still in flight so
@@ -1542,7 +1583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (u < 0) return 0;
       const Work w = map_work<DECODE>(a, u);
       TileWalker tw;
-      return walker_init<DECODE, BM>(a, w, tw);
+      return walker_init<DECODE, BM, kDescWalk<DECODE, MOD>>(a, w, tw);
     };
     // Turn token between two issuing warps: batch b of subtile 1 follows
     // batch b of subtile 0, batch b + 1 of subtile 0 follows batch b of
@@ -1672,7 +1713,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       u_next = r < rounds ? unit_of(r) : -1;
       if (u_next >= 0) {
         w_next = map_work<DECODE>(a, u_next);
-        n_next = walker_init<DECODE, BM>(a, w_next, tw_next);
+        n_next = walker_init<DECODE, BM, kDescWalk<DECODE, MOD>>(a, w_next, tw_next);
       }
     };
     setup(0);
@@ -1703,7 +1744,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (DECODE)
           tw.t += 2;
         else
-          walker_next<BM>(tw);
+          walker_next<BM, kDescWalk<DECODE, MOD>>(tw);
       }
       if (!ok) break;
       setup(r + 1);

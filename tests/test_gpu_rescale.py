@@ -3,7 +3,7 @@ exact powers of two, so a tile's (or half tile's) max exceeds the row's
 reference by far more than the rescale threshold. This drives the paths that
 redo P against the new max and rescale O: within a tile (first-chunk guess
 too low), across tiles, in the whole-tile schedule (no score mod, decode)
-and in the half-tile schedule (softcap)."""
+and in the half-tile schedule (softcap, ALiBi)."""
 import numpy as np
 import pytest
 
@@ -42,6 +42,10 @@ def prefill_case(Sq, Skv, Hq, Hkv, D, seed, ranges, **kw):
         okw.update(mask=W.MASK_WINDOW, window=kw["window"])
     if kw.get("softcap") is not None:
         okw.update(mod=W.MOD_SOFTCAP, softcap=kw["softcap"])
+    alibi = kw.pop("alibi_np", None)
+    if alibi is not None:
+        okw.update(mod=W.MOD_ALIBI, alibi=alibi)
+        kw["alibi_slopes"] = torch.from_numpy(alibi).cuda()
     o_ref, lse_ref = oracle.attn(q, k, v, **okw)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     o, lse = ea.attn_fwd(dev_bf16(q), dev_bf16(k), dev_bf16(v), status=status, **kw)
@@ -67,6 +71,12 @@ def test_growing_max_head_dim_64():
 
 def test_growing_max_softcap_half_tiles():
     prefill_case(700, 700, 4, 2, 128, 231, GROWING, softcap=30.0, window=(1023, 0))
+
+
+def test_growing_max_alibi_half_tiles():
+    # ALiBi folds the reference max into its bias: the redo must undo that
+    prefill_case(700, 700, 4, 2, 128, 235, GROWING, causal=True, alibi_np=W.alibi_slopes(4))
+    prefill_case(500, 900, 4, 1, 64, 236, GROWING, alibi_np=W.alibi_slopes(4))
 
 
 def test_growing_max_decode():
