@@ -18,9 +18,9 @@
 // twice as long as the two GEMMs of a tile, so a single query tile per CTA
 // would leave the tensor cores idle ("FlexAttention + FlashAttention-4" talk,
 // the two-Q-tile ping-pong pipeline). MMA order per step, whole tiles
-// (decode, and prefill without a score mod):
+// (decode, and prefill without the softcap):
 //   PV(0, j) QK(0, j+1) PV(1, j) QK(1, j+1)
-// Prefill with a score mod hands tiles over in key halves a (keys 0-63) and
+// Prefill with the softcap hands tiles over in key halves a (keys 0-63) and
 // b (keys 64-127), see "prefill, half tiles" below:
 //   PVa(0) QKa(0) PVa(1) QKa(1) PVb(0) QKb(0) PVb(1) QKb(1)
 // TMEM (512 columns): S0 | S1 | O0 | O1. P (bf16) overwrites part of its S
@@ -321,6 +321,10 @@ struct TileWalker {
 // hold the largest biases and later ones rarely exceed them.
 template <bool DECODE, int MOD>
 constexpr bool kDescWalk = !DECODE && MOD == MOD_ALIBI;
+// Prefill softmax with ALiBi: minus the row's reference max joins the bias,
+// so the biased scores come out as exponents (one packed op per pair fewer).
+template <int MOD>
+constexpr bool kFoldRef = MOD == MOD_ALIBI;
 constexpr int kWalkEnd = 0x7fffffff;  // walker_peek past the last tile
 
 // Head i of an ascending list of n entries, taken from the front or the back.
@@ -788,7 +792,7 @@ __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, in
 // the exponentials follow once the max is known.
 template <bool DECODE, int MOD, bool MASKED, bool BM>
 __device__ __forceinline__ float prepare_tile(const FwdArgs& a, const Work& w, int s, int row, int t, uint32_t tS,
-                                              float* x) {
+                                              float* x, float off = 0.0f) {
   const float NEG_INF = -__int_as_float(0x7f800000);
   MaskRow mr;
   if constexpr (MASKED) mr = mask_row<DECODE, BM>(a, w, s, row, t);
@@ -799,7 +803,7 @@ __device__ __forceinline__ float prepare_tile(const FwdArgs& a, const Work& w, i
   reg_fence_f<128>(x);
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    if constexpr (MOD != MOD_NONE) mod_chunk<DECODE, MOD>(a, w, s, row, t, c, x + 32 * c);
+    if constexpr (MOD != MOD_NONE) mod_chunk<DECODE, MOD>(a, w, s, row, t, c, x + 32 * c, off);
     if constexpr (MASKED) (void)mask_chunk<DECODE, BM>(a, mr, t, c, x + 32 * c);
     mc = fmaxf(mc, chunk_max(x + 32 * c));
   }
@@ -861,6 +865,7 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
   float mt;
   const bool have_ref = !first && __all_sync(0xffffffffu, st.m != NEG_INF);
   const float nmu0 = have_ref ? -st.m : 0.0f;
+  float xref = 0.0f;  // the scores in x are relative to this (prefill ALiBi with a reference max)
   bool guessed = false;
   if (cls == 0) {
 #pragma unroll
@@ -894,19 +899,26 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
     guessed = true;
   } else {
     // Scores (with mods and mask) first; the exponentials follow against the
-    // reference max when there is one, else in the slow path below.
+    // reference max when there is one, else in the slow path below. With
+    // ALiBi in prefill the reference rides in the bias (x relative to xref).
+    constexpr bool kFold = kFoldRef<MOD> && !DECODE;
+    const float off = (kFold && have_ref) ? -st.m : 0.0f;
+    xref = -off;
     float mc;
     if (cls == 2)
-      mc = prepare_tile<DECODE, MOD, false, BM>(a, w, s, row, t, tS, x);
+      mc = prepare_tile<DECODE, MOD, false, BM>(a, w, s, row, t, tS, x, off);
     else
-      mc = prepare_tile<DECODE, MOD, true, BM>(a, w, s, row, t, tS, x);
-    mt = mc * mult;
+      mc = prepare_tile<DECODE, MOD, true, BM>(a, w, s, row, t, tS, x, off);
+    mt = mc * mult + xref;
     if (have_ref) {
       const float2 NMU = make_float2(nmu0, nmu0);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
-        exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
+        if constexpr (kFold)
+          exp_chunk<false>(x + 32 * c, MULT, NMU, pk, acc0, acc1);
+        else
+          exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
         tmem_st16(tS + 16 * c, pk);
       }
     }
@@ -919,7 +931,7 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
     const float m_new = fmaxf(st.m, mt);
     alpha = (m_new == NEG_INF || st.m == NEG_INF) ? (st.m == NEG_INF ? 0.0f : 1.0f) : ex2(st.m - m_new);
     st.m = m_new;
-    const float nmu = (m_new == NEG_INF) ? 0.0f : -m_new;
+    const float nmu = (m_new == NEG_INF) ? 0.0f : xref - m_new;
     const float2 NMU = make_float2(nmu, nmu);
     acc0 = acc1 = make_float2(0.f, 0.f);
     tmem_st_wait();  // the optimistic P stores (if any) land before they are overwritten
@@ -957,15 +969,14 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
 }
 
 // ---------------------------------------------------------------- prefill, half tiles
-// Kernels with a score mod (softcap, ALiBi) hand each key tile to the tensor
-// pipe in two halves; their softmax is long enough that overlapping it with
-// the MMAs pays for the extra hand-offs (+6-8 % measured). Without a mod the
-// whole-tile schedule is faster (the half schedule measured 5 % slower).
+// The softcap kernel hands each key tile to the tensor pipe in two halves:
+// its softmax (tanh series, then exponentials) is long enough that
+// overlapping it with the MMAs pays for the extra hand-offs (whole tiles
+// measured 11 % slower). Without a mod, and with ALiBi since its tiles are
+// walked from the diagonal back (no rescales), whole tiles are faster (the
+// half schedule measured 5 % and 7 % slower).
 template <bool DECODE, int MOD>
-constexpr bool kHalfTiles = !DECODE && MOD != MOD_NONE && MOD != MOD_RELU;
-// Half-tile softmax: fold minus the reference max into the ALiBi bias.
-template <int MOD>
-constexpr bool kFoldRef = MOD == MOD_ALIBI;
+constexpr bool kHalfTiles = !DECODE && MOD == MOD_SOFTCAP;
 
 // With half tiles: P for keys
 // 0-63 goes to S(s) columns [0, 32) and P for keys 64-127 to [64, 96), so:
@@ -1556,7 +1567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (last) mma_commit(&bar.q_empty);
       mma_commit(&bar.k_empty[slot]);
     };
-    // Prefill with a score mod: QK^T and PV in key halves (see "prefill, half tiles").
+    // Prefill with the softcap: QK^T and PV in key halves (see "prefill, half tiles").
     constexpr uint32_t idesc_qk_half = idesc_bf16_f32(128, 64, 0, 0);
     constexpr uint32_t kHalfKeyUnits = (64 * 128) >> 4;  // 64 K rows of a 128-byte SW128 box
     auto qk_half_mmas = [&](int s, int slot, int h, bool last) {

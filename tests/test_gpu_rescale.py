@@ -3,7 +3,7 @@ exact powers of two, so a tile's (or half tile's) max exceeds the row's
 reference by far more than the rescale threshold. This drives the paths that
 redo P against the new max and rescale O: within a tile (first-chunk guess
 too low), across tiles, in the whole-tile schedule (no score mod, decode)
-and in the half-tile schedule (softcap, ALiBi)."""
+and in the half-tile schedule (softcap), and with ALiBi."""
 import numpy as np
 import pytest
 
@@ -73,8 +73,8 @@ def test_growing_max_softcap_half_tiles():
     prefill_case(700, 700, 4, 2, 128, 231, GROWING, softcap=30.0, window=(1023, 0))
 
 
-def test_growing_max_alibi_half_tiles():
-    # ALiBi folds the reference max into its bias: the redo must undo that
+def test_growing_max_alibi():
+    # ALiBi tiles are walked from the diagonal back; the max still grows here
     prefill_case(700, 700, 4, 2, 128, 235, GROWING, causal=True, alibi_np=W.alibi_slopes(4))
     prefill_case(500, 900, 4, 1, 64, 236, GROWING, alibi_np=W.alibi_slopes(4))
 
