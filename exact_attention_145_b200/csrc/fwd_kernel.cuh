@@ -1035,7 +1035,7 @@ __device__ __forceinline__ float stream_half(const FwdArgs& a, const Work& w, in
 // exponentials once the reference is known.
 template <int MOD, bool MASKED, bool BM>
 __device__ __forceinline__ float prepare_half(const FwdArgs& a, const Work& w, int s, int row, int t, uint32_t tS,
-                                              int h, float* x, float off) {
+                                              int h, float* x) {
   const float NEG_INF = -__int_as_float(0x7f800000);
   MaskRow mr;
   if constexpr (MASKED) mr = mask_row<false, BM>(a, w, s, row, t);
@@ -1048,7 +1048,7 @@ __device__ __forceinline__ float prepare_half(const FwdArgs& a, const Work& w, i
 #pragma unroll
   for (int cc = 0; cc < 2; ++cc) {
     const int c = 2 * h + cc;
-    if constexpr (MOD != MOD_NONE) mod_chunk<false, MOD>(a, w, s, row, t, c, x + 32 * cc, off);
+    if constexpr (MOD != MOD_NONE) mod_chunk<false, MOD>(a, w, s, row, t, c, x + 32 * cc);
     if constexpr (MASKED) (void)mask_chunk<false, BM>(a, mr, t, c, x + 32 * cc);
     mc = fmaxf(mc, chunk_max(x + 32 * cc));
   }
@@ -1104,7 +1104,6 @@ __device__ __forceinline__ bool softmax_step_halves(const FwdArgs& a, const Work
     float x[64];
     float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
     float mh;
-    float xref = 0.0f;  // the scores in x are relative to this (ALiBi with a reference max)
     const bool have_ref = __all_sync(0xffffffffu, st.m != NEG_INF);
     bool guessed = false;
     if (cls == 0) {
@@ -1131,26 +1130,18 @@ __device__ __forceinline__ bool softmax_step_halves(const FwdArgs& a, const Work
       }
       guessed = true;
     } else {
-      // ALiBi with a reference max: minus the reference joins the bias, so
-      // the half's scores come out as exponents (one packed op per pair
-      // fewer); xref is what they are relative to.
-      const float off = (kFoldRef<MOD> && have_ref) ? -st.m : 0.0f;
-      xref = -off;
       float mc;
       if (cls == 2)
-        mc = prepare_half<MOD, false, BM>(a, w, s, row, t, tS, h, x, off);
+        mc = prepare_half<MOD, false, BM>(a, w, s, row, t, tS, h, x);
       else
-        mc = prepare_half<MOD, true, BM>(a, w, s, row, t, tS, h, x, off);
-      mh = mc * mult + xref;
+        mc = prepare_half<MOD, true, BM>(a, w, s, row, t, tS, h, x);
+      mh = mc * mult;
       if (have_ref) {
         const float2 NMU = make_float2(-st.m, -st.m);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
-          if constexpr (kFoldRef<MOD>)
-            exp_chunk<false>(x + 32 * c, MULT, NMU, pk, acc0, acc1);
-          else
-            exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
+          exp_chunk(x + 32 * c, MULT, NMU, pk, acc0, acc1);
           tmem_st16(tS + 64 * h + 16 * c, pk);
         }
       }
@@ -1161,7 +1152,7 @@ __device__ __forceinline__ bool softmax_step_halves(const FwdArgs& a, const Work
       const float m_new = fmaxf(st.m, mh);
       alpha = (m_new == NEG_INF || st.m == NEG_INF) ? (st.m == NEG_INF ? 0.0f : 1.0f) : ex2(st.m - m_new);
       st.m = m_new;
-      const float nmu = (m_new == NEG_INF) ? 0.0f : xref - m_new;
+      const float nmu = (m_new == NEG_INF) ? 0.0f : -m_new;
       const float2 NMU = make_float2(nmu, nmu);
       acc0 = acc1 = make_float2(0.f, 0.f);
       tmem_st_wait();  // the optimistic P stores land before they are overwritten
