@@ -931,7 +931,7 @@ __device__ __forceinline__ void softmax_step(const FwdArgs& a, const Work& w, in
     const float m_new = fmaxf(st.m, mt);
     alpha = (m_new == NEG_INF || st.m == NEG_INF) ? (st.m == NEG_INF ? 0.0f : 1.0f) : ex2(st.m - m_new);
     st.m = m_new;
-    const float nmu = (m_new == NEG_INF) ? 0.0f : xref - m_new;
+    const float nmu = (m_new == NEG_INF) ? 0.0f : (kFoldRef<MOD> && !DECODE ? xref - m_new : -m_new);
     const float2 NMU = make_float2(nmu, nmu);
     acc0 = acc1 = make_float2(0.f, 0.f);
     tmem_st_wait();  // the optimistic P stores (if any) land before they are overwritten
