@@ -787,9 +787,10 @@ __device__ __forceinline__ float stream_tile(const FwdArgs& a, const Work& w, in
   return mc;
 }
 
-// First tile of a row: loads the scores chunk by chunk (the next chunk in
-// flight while this one gets its mods and mask) and returns the raw row max;
-// the exponentials follow once the max is known.
+// Scores of a whole tile with mods and mask (all four chunks requested from
+// TMEM before one wait); returns the row max of the modded scores. The
+// exponentials follow once the reference is known. off is added to the ALiBi
+// bias (minus the row's reference max in prefill, else 0).
 template <bool DECODE, int MOD, bool MASKED, bool BM>
 __device__ __forceinline__ float prepare_tile(const FwdArgs& a, const Work& w, int s, int row, int t, uint32_t tS,
                                               float* x, float off = 0.0f) {
